@@ -1,0 +1,85 @@
+"""Scalar brute force of the BSFA definition (test infrastructure only).
+
+A second statement of the same definition as ``bsfa_oracle``, written as plain
+Python loops with no BLAS and no vectorisation, for tiny inputs only. It does
+not reuse the oracle's geometry helpers: block visibility, the forced
+("diagonal") blocks and the block maxima are found here by enumerating the
+(query, key) pairs of each block.
+
+Source: "Block Sparse Flash Attention" (paperpeel.com/paper/2512.07011),
+§4.1 "Gating Mechanism" (gate on the exact block maximum; diagonal blocks bypass
+it), §4.4 (skipped blocks stay out of the running statistics), App. B.2 (scaled
+scores, softmax), App. B.3 (bidirectional case).
+"""
+from __future__ import annotations
+
+import math
+
+
+def _is_valid(r: int, c: int, causal: bool) -> bool:
+    return c <= r if causal else True
+
+
+def brute_forward(q, k, v, tau, Bq: int, Bk: int, causal: bool):
+    """q: float [B][N][Hq][D]; k, v: float [B][N][Hkv][D]; tau: [Hq].
+
+    Returns (out [B][N][Hq][D], lse [B][Hq][N], codes {(b, hq, i, j): code}).
+    """
+    B, N, Hq, D = len(q), len(q[0]), len(q[0][0]), len(q[0][0][0])
+    Hkv = len(k[0][0])
+    per_kv = Hq // Hkv
+    inv = 1.0 / math.sqrt(D)
+    mq = (N + Bq - 1) // Bq
+    mkv = (N + Bk - 1) // Bk
+    out = [[[[0.0] * D for _ in range(Hq)] for _ in range(N)] for _ in range(B)]
+    lse = [[[0.0] * N for _ in range(Hq)] for _ in range(B)]
+    codes = {}
+    for b in range(B):
+        for hq in range(Hq):
+            g = hq // per_kv
+            s = [[0.0] * N for _ in range(N)]
+            for r in range(N):
+                for c in range(N):
+                    acc = 0.0
+                    for d in range(D):
+                        acc += q[b][r][hq][d] * k[b][c][g][d]
+                    s[r][c] = acc * inv
+            for i in range(mq):
+                rows = range(i * Bq, min((i + 1) * Bq, N))
+                for j in range(mkv):
+                    cols = range(j * Bk, min((j + 1) * Bk, N))
+                    any_valid = False
+                    any_invalid = False
+                    best = -math.inf
+                    for r in rows:
+                        for c in cols:
+                            if _is_valid(r, c, causal):
+                                any_valid = True
+                                if s[r][c] > best:
+                                    best = s[r][c]
+                            else:
+                                any_invalid = True
+                    if not any_valid:
+                        codes[(b, hq, i, j)] = 3
+                        continue
+                    if causal:
+                        forced = any_invalid
+                    else:
+                        forced = any(c in rows for c in cols)
+                    if forced:
+                        codes[(b, hq, i, j)] = 2
+                    elif best >= tau[hq]:
+                        codes[(b, hq, i, j)] = 1
+                    else:
+                        codes[(b, hq, i, j)] = 0
+            for r in range(N):
+                i = r // Bq
+                kept = [c for c in range(N)
+                        if _is_valid(r, c, causal) and codes[(b, hq, i, c // Bk)] in (1, 2)]
+                m = max(s[r][c] for c in kept)
+                weights = [math.exp(s[r][c] - m) for c in kept]
+                total = sum(weights)
+                for d in range(D):
+                    out[b][r][hq][d] = sum(w * v[b][c][g][d] for w, c in zip(weights, kept)) / total
+                lse[b][hq][r] = m + math.log(total)
+    return out, lse, codes
