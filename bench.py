@@ -1,0 +1,401 @@
+#!/usr/bin/env python
+"""Throughput of the BSFA prefill forward (one attention layer per step) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config c2] [--skip 0.5]
+    python bench.py --impl reference ...      # the CPU oracle on a bounded sample
+
+A step is one ``bsfa_forward`` call over every head of the layer (all rows of the
+hot path: QK^T, block maxima, gate, online softmax, PV for kept blocks,
+epilogue), on synthetic inputs already resident in HBM; L2 is flushed with a
+256 MB memset between steps, outside the timed events. The metric is
+dense-equivalent TFLOP/s: the FLOPs the same tiles would cost with every
+visible block kept (2*Bq*Bk*D for QK^T plus 2*Bq*Bk*D for PV per visible tile),
+divided by the kernel time. Executed TFLOP/s counts PV only for kept tiles.
+The same kernel at tau = -inf gives the dense comparator. ``e2e`` repeats the
+measurement through the host-buffer call (pinned host inputs copied in, out and
+lse copied back, inside the timed region).
+
+For N > 1 (torchrun) every rank runs its own copy of the layer (independent
+problems, no data-path collective): weak scaling, value = all ranks' FLOPs over
+the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from threshold_gated_block_b200.inputs import CONFIGS, make_inputs, sample_tiles  # noqa: E402
+
+METRIC = "prefill-attention TFLOP/s (dense-equivalent)"
+UNIT = "TFLOP/s"
+TAUS = os.path.join(ROOT, "tests", "golden", "taus.json")
+PEAKS = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC = os.path.join(ROOT, "profiles", "bsfa_fwd_c2_traffic.txt")
+KERNEL_SOURCES = ["ptx.cuh", "bsfa_fwd_kernel.cuh", "bsfa_launch.cuh", "bsfa_fwd_d64.cu", "bsfa_fwd_d128.cu",
+                  "bsfa_api.cu"]
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="c2")
+    ap.add_argument("--skip", type=float, default=None, help="target skip fraction (a stored calibration)")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU-oracle baseline")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def workload(args):
+    cfg = CONFIGS[args.config]
+    p = cfg.skips[0] if args.skip is None else args.skip
+    with open(TAUS) as f:
+        taus = json.load(f)[cfg.name]["taus"][str(float(p))]
+    return cfg, p, taus
+
+
+def config_record(cfg, p, achieved=None):
+    rec = {"workload": f"{cfg.name}: {cfg.description}", "B": cfg.B, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "D": cfg.D,
+           "N": cfg.N, "Bq": cfg.Bq, "Bk": cfg.Bk, "causal": cfg.causal, "inputs": cfg.kind,
+           "target_skip": p, "l2": "flushed between steps (256 MB memset outside the timed events)"}
+    if achieved is not None:
+        rec["achieved_skip"] = achieved
+    return rec
+
+
+def tile_flop(cfg) -> float:
+    return 2.0 * cfg.Bq * cfg.Bk * cfg.D
+
+
+def mask_flops(mask: np.ndarray, cfg):
+    """(executed, dense-equivalent) FLOPs of one layer from the block codes."""
+    visited = int((mask != 3).sum())
+    kept = int(np.isin(mask, (1, 2)).sum())
+    f = tile_flop(cfg)
+    return (visited + kept) * f, 2 * visited * f
+
+
+def cpu_cores():
+    try:
+        from threadpoolctl import threadpool_info
+        n = max((i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"), default=0)
+        if n:
+            return n
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def oracle_sample(cfg, x, taus, budget_s, tiles):
+    """Run the oracle on sampled tiles until the budget is spent: (dense FLOPs, seconds, tiles)."""
+    from oracle import bsfa_oracle as O
+    tau = np.asarray(taus, dtype=np.float64)
+    f = tile_flop(cfg)
+    flops, done, t0 = 0.0, 0, time.perf_counter()
+    for (b, h, i) in tiles:
+        t = O.forward_tile(x["q"], x["k"], x["v"], tau, b, h, i, cfg.Bq, cfg.Bk, cfg.causal)
+        flops += 2 * int((t["codes"] != O.CODE_INVISIBLE).sum()) * f
+        done += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    return flops, time.perf_counter() - t0, done
+
+
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "threshold_gated_block_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(cfg):
+    """DRAM bytes per launch from the committed ncu summary, if it matches this kernel and workload."""
+    if not os.path.exists(TRAFFIC):
+        return None
+    kv = {}
+    with open(TRAFFIC) as f:
+        for line in f:
+            if ":" in line:
+                k, v = line.split(":", 1)
+                kv[k.strip()] = v.strip()
+    if kv.get("kernel_hash") != kernel_hash() or kv.get("config") != cfg.name:
+        return None
+    try:
+        return float(kv["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the GPU works."""
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.hw_slowdown",
+              "clocks_event_reasons.hw_thermal_slowdown", "clocks_event_reasons.sw_thermal_slowdown",
+              "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, device_index: int, bus_id: str | None):
+        self.proc = None
+        target = bus_id or str(device_index)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={target}", "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.splitlines():
+            parts = [s.strip() for s in line.split(",")]
+            if len(parts) != len(self.FIELDS):
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- reference arm (CPU oracle)
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    cfg, p, taus = workload(args)
+    x = make_inputs(cfg)
+    tiles = sample_tiles(cfg, 4096, seed=cfg.seed + 5)
+    rng = np.random.default_rng(0)
+    rng.shuffle(tiles)
+    per_step = max(0.05, min(2.0, 150.0 / max(args.steps + args.warmup, 1)))
+    pos = 0
+    for _ in range(args.warmup):
+        _, _, n = oracle_sample(cfg, x, taus, per_step, tiles[pos:] + tiles[:pos])
+        pos = (pos + n) % len(tiles)
+    tot_f, tot_t, tot_n = 0.0, 0.0, 0
+    for _ in range(args.steps):
+        f, t, n = oracle_sample(cfg, x, taus, per_step, tiles[pos:] + tiles[:pos])
+        pos = (pos + n) % len(tiles)
+        tot_f, tot_t, tot_n = tot_f + f, tot_t + t, tot_n + n
+    value = tot_f / tot_t / 1e12
+    cores = cpu_cores()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_record(cfg, p),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"{tot_n} query tiles of {cfg.name} (about {per_step:.2f} s of oracle work per "
+                                   f"step), dense-equivalent FLOPs of those tiles"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+
+    from threshold_gated_block_b200 import bsfa
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=180), device_id=dev)
+    bsfa.load()
+
+    cfg, p, taus = workload(args)
+    x = make_inputs(cfg)
+    to_dev = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+    q, k, v = to_dev(x["q"]), to_dev(x["k"]), to_dev(x["v"])
+    tau = torch.tensor(taus, dtype=torch.float32, device=dev)
+    tau_dense = torch.full_like(tau, float("-inf"))
+    out = torch.empty_like(q)
+    lse = torch.empty((cfg.B, cfg.Hq, cfg.N), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(t):
+        st = bsfa.bsfa_forward(q, k, v, t, out, lse, None, cfg.B, cfg.Hq, cfg.Hkv, cfg.N, cfg.D, cfg.Bq, cfg.Bk,
+                               cfg.causal, stream)
+        if st != bsfa.BSFA_OK:
+            raise RuntimeError(bsfa.bsfa_last_error())
+
+    # Block codes of this layer (untimed) give the executed and dense-equivalent FLOPs.
+    _, _, mask = bsfa.forward(q, k, v, tau, Bq=cfg.Bq, Bk=cfg.Bk, causal=cfg.causal, want_lse=False, want_mask=True)
+    m = mask.cpu().numpy()
+    del mask
+    exec_flops, dense_flops = mask_flops(m, cfg)
+    gated = np.isin(m, (0, 1))
+    achieved_skip = float((m == 0).sum() / max(gated.sum(), 1))
+    kv_bytes = cfg.B * cfg.N * cfg.Hkv * cfg.D * 2
+
+    def timed(t, steps):
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        for i in range(steps):
+            flush.zero_()
+            starts[i].record(stream)
+            step(t)
+            ends[i].record(stream)
+        torch.cuda.synchronize(dev)
+        return [s.elapsed_time(e) for s, e in zip(starts, ends)]
+
+    def barrier():
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(val: float) -> float:
+        if world == 1:
+            return val
+        t = torch.tensor([val], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    props = torch.cuda.get_device_properties(dev)
+    bus = None
+    if hasattr(props, "pci_bus_id"):
+        bus = f"{getattr(props, 'pci_domain_id', 0):08X}:{props.pci_bus_id:02X}:{getattr(props, 'pci_device_id', 0):02X}.0"
+    sampler = ClockSampler(local, bus)
+    time.sleep(0.3)
+
+    for _ in range(args.warmup):
+        step(tau)
+    barrier()
+    times = timed(tau, args.steps)                     # the timed region: exactly K steps
+    barrier()
+    t_total = max_over_ranks(sum(times))
+    ms = t_total / args.steps
+
+    # Dense comparator: the same kernel at tau = -inf.
+    for _ in range(args.warmup):
+        step(tau_dense)
+    barrier()
+    dense_ms = max_over_ranks(sum(timed(tau_dense, args.steps))) / args.steps
+
+    e2e = None
+    if not args.no_e2e:
+        hq = torch.empty(q.shape, dtype=torch.bfloat16, pin_memory=True)
+        hk = torch.empty(k.shape, dtype=torch.bfloat16, pin_memory=True)
+        hv = torch.empty(v.shape, dtype=torch.bfloat16, pin_memory=True)
+        ht = torch.tensor(taus, dtype=torch.float32).pin_memory()
+        hq.copy_(q.cpu()); hk.copy_(k.cpu()); hv.copy_(v.cpu())
+        bufs = bsfa.device_buffers(q.shape, k.shape, dev)
+        ke = max(3, min(args.steps, 30))
+        for _ in range(max(1, min(args.warmup, 3))):
+            bsfa.forward_host(hq, hk, hv, ht, Bq=cfg.Bq, Bk=cfg.Bk, causal=cfg.causal, device=dev, stream=stream,
+                              bufs=bufs)
+        barrier()
+        et = []
+        for _ in range(ke):
+            s0 = torch.cuda.Event(enable_timing=True)
+            s1 = torch.cuda.Event(enable_timing=True)
+            s0.record(stream)
+            bsfa.forward_host(hq, hk, hv, ht, Bq=cfg.Bq, Bk=cfg.Bk, causal=cfg.causal, device=dev, stream=stream,
+                              bufs=bufs)
+            s1.record(stream)
+            torch.cuda.synchronize(dev)
+            et.append(s0.elapsed_time(s1))
+        e2e_ms = max_over_ranks(sum(et)) / ke
+        h2d = (hq.numel() + hk.numel() + hv.numel()) * 2 + ht.numel() * 4
+        d2h = bufs["out_host"].numel() * 2 + bufs["lse_host"].numel() * 4
+        e2e = {"value": world * dense_flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": ke}
+
+    clocks = sampler.stop()
+    status = bsfa.bsfa_get_status(stream)
+    if status != bsfa.BSFA_OK:
+        raise RuntimeError(f"device status: {bsfa.bsfa_last_error()}")
+
+    exec_tflops = exec_flops / (ms * 1e-3) / 1e12
+    dense_tflops = dense_flops / (ms * 1e-3) / 1e12
+    peak, peak_src = FALLBACK_BF16_TFLOPS, "fallback"
+    if os.path.exists(PEAKS):
+        with open(PEAKS) as f:
+            peaks = json.load(f)
+        if peaks.get("bf16_tflops"):
+            peak, peak_src = float(peaks["bf16_tflops"]), "measured (MEASURED_PEAKS.json bf16_tflops, burst)"
+    traffic = measured_traffic(cfg)
+
+    line = None
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": world * dense_tflops, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": config_record(cfg, p, achieved_skip),
+            "exec_tflops": world * exec_tflops, "dense_equiv_tflops": world * dense_tflops,
+            "ms_per_layer": ms, "dense_ms_per_layer": dense_ms, "speedup_vs_dense": dense_ms / ms,
+            "exec_flops_per_layer": exec_flops, "dense_flops_per_layer": dense_flops,
+            "roofline": {"bound": "tensor", "achieved": exec_tflops, "peak": peak, "unit": UNIT,
+                         "frac": exec_tflops / peak, "traffic": traffic, "peak_source": peak_src,
+                         "kernel": "bsfa_fwd_kernel", "kv_bytes_per_head_tensor": kv_bytes},
+            "gpu_launches": args.steps,
+            "clocks": clocks,
+        }
+        if e2e is not None:
+            line["e2e"] = e2e
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        if world == 1:
+            budget = args.cpu_seconds
+            tiles = sample_tiles(cfg, 4096, seed=cfg.seed + 5)
+            np.random.default_rng(0).shuffle(tiles)
+            f, t, n = oracle_sample(cfg, x, taus, budget, tiles)
+            line["cpu_baseline"] = {"value": f / t / 1e12, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+                                    "sample": f"{n} seeded query tiles of {cfg.name} (about {t:.1f} s of oracle "
+                                              f"work), dense-equivalent FLOPs of those tiles"}
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

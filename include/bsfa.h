@@ -1,0 +1,102 @@
+/*
+ * bsfa.h - C ABI of the B200 (sm_100a) Block Sparse Flash Attention prefill forward.
+ *
+ * The operation ("Block Sparse Flash Attention", §4 Method, §4.1 Gating
+ * Mechanism, §4.4 Algorithm and Implementation, App. B.2): tiled online-softmax
+ * attention that computes every score S = Q K^T / sqrt(d) exactly. For each
+ * (query tile i, key block j) it takes the block maximum s_max(i,j) over the
+ * valid entries; when s_max(i,j) < tau[h] the block's values are not loaded, the
+ * PV product is not run and the running statistics (m, l, O) are not updated.
+ * Diagonal blocks bypass the gate. The result is therefore the softmax over each
+ * query tile's kept key set.
+ *
+ * Definitions used by every entry point:
+ *   - Query tile i holds rows [i*Bq, (i+1)*Bq); key block j holds keys [j*Bk, (j+1)*Bk).
+ *   - Causal: key c is valid for query r when c <= r. A block is visible when some
+ *     entry is valid; it is diagonal (gate bypassed) when it is visible and also
+ *     holds an invalid entry. Non-causal ("bidirectional", App. B.3): the diagonal
+ *     blocks are those whose key range overlaps the tile's query range.
+ *   - tau is in units of the scaled score q.k/sqrt(d); a block whose maximum
+ *     equals tau is kept. tau = -INFINITY gives dense attention.
+ *   - GQA: query head h reads KV head h / (Hq / Hkv).
+ *
+ * Thread safety: entry points may be called from several host threads; calls on
+ * the same stream are ordered by the stream. The library allocates nothing per
+ * call; it keeps one device status word per device.
+ */
+#ifndef BSFA_H_
+#define BSFA_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  BSFA_OK = 0,
+  BSFA_ERR_INVALID_ARG = 1,     /* null pointer, non-positive size, Hq % Hkv != 0, misaligned pointer */
+  BSFA_ERR_UNSUPPORTED = 2,     /* D, Bq, Bk or N outside the supported set, or no sm_100 device */
+  BSFA_ERR_CUDA = 3,            /* a CUDA runtime or driver call failed (see bsfa_last_error) */
+  BSFA_ERR_DEVICE_TIMEOUT = 4   /* a kernel gave up on a bounded wait (reported by bsfa_get_status) */
+} bsfa_status;
+
+/*
+ * bsfa_forward - BSFA prefill forward for a batch of heads, asynchronous on `stream`.
+ *
+ *   q          bf16 [B, N, Hq,  D], contiguous, device memory, 16-byte aligned (read)
+ *   k          bf16 [B, N, Hkv, D], contiguous, device memory, 16-byte aligned (read)
+ *   v          bf16 [B, N, Hkv, D], contiguous, device memory, 16-byte aligned (read; only
+ *              the blocks some query tile keeps are loaded)
+ *   tau        fp32 [Hq], device memory: one threshold per query head (§4.1; the paper's
+ *              table indexed by layer, head and position is reduced to one value per head)
+ *   out        bf16 [B, N, Hq, D], contiguous, device memory, 16-byte aligned (written)
+ *   lse        fp32 [B, Hq, N], device memory, natural-log logsumexp over each row's kept
+ *              set (written); NULL skips it
+ *   block_mask uint8 [B, Hq, N/Bq, N/Bk], device memory (written); NULL turns the debug
+ *              output off. Codes: 0 skipped by the gate, 1 kept by the gate, 2 diagonal
+ *              (forced keep), 3 not visible. The library fills it with 3 first.
+ *   B, Hq, Hkv, N, D   sizes; Hq % Hkv == 0
+ *   Bq, Bk     query-tile and key-block sizes (the paper's B_M and B_N)
+ *   causal     nonzero for causal prefill, zero for bidirectional attention
+ *   stream     a cudaStream_t (NULL = the legacy default stream)
+ *
+ * Supported: D in {64, 128}; Bq, Bk in {64, 128}; N a positive multiple of 128;
+ * an sm_100 device. The caller owns every buffer; results are valid once the
+ * stream has reached the call. Returns BSFA_OK once the kernel is enqueued;
+ * argument errors are returned before any CUDA call is made. A kernel that gives
+ * up on a bounded internal wait leaves `out` undefined and sets the device
+ * status word that bsfa_get_status reports.
+ */
+bsfa_status bsfa_forward(const void* q, const void* k, const void* v, const float* tau, void* out, float* lse,
+                         uint8_t* block_mask, int B, int Hq, int Hkv, int N, int D, int Bq, int Bk, int causal,
+                         void* stream);
+
+/*
+ * bsfa_validate - the shape checks of bsfa_forward, host only (no CUDA call).
+ * Returns BSFA_OK, BSFA_ERR_INVALID_ARG or BSFA_ERR_UNSUPPORTED.
+ */
+bsfa_status bsfa_validate(int B, int Hq, int Hkv, int N, int D, int Bq, int Bk, int causal);
+
+/*
+ * bsfa_get_status - synchronise `stream`, then read and clear the device status
+ * word of the current device. Returns BSFA_ERR_DEVICE_TIMEOUT when a kernel gave
+ * up on a bounded wait since the last call, BSFA_ERR_CUDA when the
+ * synchronisation itself failed, else BSFA_OK.
+ */
+bsfa_status bsfa_get_status(void* stream);
+
+/* bsfa_status_string - a static, human-readable name for a status code. */
+const char* bsfa_status_string(bsfa_status s);
+
+/*
+ * bsfa_last_error - details of the last failure on the calling host thread
+ * (a static thread-local buffer, valid until the thread's next call).
+ */
+const char* bsfa_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BSFA_H_ */

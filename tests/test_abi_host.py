@@ -1,0 +1,73 @@
+"""The C ABI without a GPU: the library loads, exports what include/bsfa.h
+declares, and rejects bad arguments before making any CUDA call."""
+import os
+import re
+import subprocess
+
+import pytest
+
+from threshold_gated_block_b200 import bsfa
+from threshold_gated_block_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return bsfa.load()
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "bsfa.h")).read()
+    return sorted(set(re.findall(r"^(?:bsfa_status|const char\*)\s+(bsfa_\w+)\(", text, flags=re.M)))
+
+
+def test_header_declares_the_binding_names():
+    assert _declared() == sorted(bsfa.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", bsfa.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (bsfa_\w+)", out))
+    for name in _declared():
+        assert name in exported, name
+        assert hasattr(lib, name)
+
+
+def test_status_strings(lib):
+    assert bsfa.bsfa_status_string(0) == "BSFA_OK"
+    assert bsfa.bsfa_status_string(4) == "BSFA_ERR_DEVICE_TIMEOUT"
+    assert bsfa.bsfa_status_string(99) == "BSFA_UNKNOWN_STATUS"
+
+
+@pytest.mark.parametrize("args,want", [
+    ((1, 32, 8, 8192, 128, 128, 128, 1), bsfa.BSFA_OK),
+    ((1, 2, 2, 512, 64, 64, 64, 1), bsfa.BSFA_OK),
+    ((2, 24, 24, 16384, 128, 64, 128, 0), bsfa.BSFA_OK),
+    ((0, 32, 8, 8192, 128, 128, 128, 1), bsfa.BSFA_ERR_INVALID_ARG),
+    ((1, 32, 7, 8192, 128, 128, 128, 1), bsfa.BSFA_ERR_INVALID_ARG),
+    ((1, -1, 1, 8192, 128, 128, 128, 1), bsfa.BSFA_ERR_INVALID_ARG),
+    ((1, 32, 8, 8192, 96, 128, 128, 1), bsfa.BSFA_ERR_UNSUPPORTED),
+    ((1, 32, 8, 8192, 128, 32, 128, 1), bsfa.BSFA_ERR_UNSUPPORTED),
+    ((1, 32, 8, 8192, 128, 128, 256, 1), bsfa.BSFA_ERR_UNSUPPORTED),
+    ((1, 32, 8, 8000, 128, 128, 128, 1), bsfa.BSFA_ERR_UNSUPPORTED),
+    ((1024, 64, 8, 65536, 128, 128, 128, 1), bsfa.BSFA_ERR_UNSUPPORTED),
+])
+def test_validate(lib, args, want):
+    assert bsfa.bsfa_validate(*args) == want
+    if want != bsfa.BSFA_OK:
+        assert bsfa.bsfa_last_error()
+
+
+def test_forward_rejects_bad_pointers_without_touching_cuda(lib):
+    shape = (1, 2, 2, 512, 64, 64, 64, 1)
+    # null q
+    assert bsfa.bsfa_forward(None, 16, 16, 16, 16, None, None, *shape, None) == bsfa.BSFA_ERR_INVALID_ARG
+    # misaligned k
+    assert bsfa.bsfa_forward(16, 24, 16, 16, 16, None, None, *shape, None) == bsfa.BSFA_ERR_INVALID_ARG
+    # misaligned lse
+    assert bsfa.bsfa_forward(16, 16, 16, 16, 16, 2, None, *shape, None) == bsfa.BSFA_ERR_INVALID_ARG
+    # unsupported shape wins before pointer checks
+    assert bsfa.bsfa_forward(None, None, None, None, None, None, None, 1, 2, 2, 500, 64, 64, 64, 1, None) \
+        == bsfa.BSFA_ERR_UNSUPPORTED

@@ -1,0 +1,175 @@
+"""Python binding of the BSFA C ABI (include/bsfa.h).
+
+Argument marshalling only: every step of the forward runs in the CUDA kernels
+of libbsfa.so. PyTorch supplies device memory and streams. There is no CPU
+fallback: if the library is missing or the device is not sm_100, calls fail
+loudly.
+
+The functions named like the C entry points (``bsfa_forward``,
+``bsfa_validate``, ``bsfa_get_status``, ``bsfa_status_string``,
+``bsfa_last_error``) take the same arguments; pointer arguments accept an int
+address, None, or a torch tensor (its ``data_ptr()``). ``forward`` and
+``forward_host`` are conveniences over ``bsfa_forward`` for torch tensors.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbsfa.so")
+
+BSFA_OK = 0
+BSFA_ERR_INVALID_ARG = 1
+BSFA_ERR_UNSUPPORTED = 2
+BSFA_ERR_CUDA = 3
+BSFA_ERR_DEVICE_TIMEOUT = 4
+
+EXPORTED = ("bsfa_forward", "bsfa_validate", "bsfa_get_status", "bsfa_status_string", "bsfa_last_error")
+
+_lib = None
+
+
+class BsfaError(RuntimeError):
+    def __init__(self, status: int, detail: str):
+        super().__init__(f"{bsfa_status_string(status)}: {detail}")
+        self.status = status
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libbsfa.so (once) and declare the C signatures."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with threshold_gated_block_b200.build.build()")
+    lib = ctypes.CDLL(path)
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    lib.bsfa_forward.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, vp]
+    lib.bsfa_forward.restype = i
+    lib.bsfa_validate.argtypes = [i] * 8
+    lib.bsfa_validate.restype = i
+    lib.bsfa_get_status.argtypes = [vp]
+    lib.bsfa_get_status.restype = i
+    lib.bsfa_status_string.argtypes = [i]
+    lib.bsfa_status_string.restype = ctypes.c_char_p
+    lib.bsfa_last_error.argtypes = []
+    lib.bsfa_last_error.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(s):
+    if s is None:
+        return None
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+# ----------------------------------------------------------------------------- C entry points
+
+def bsfa_forward(q, k, v, tau, out, lse, block_mask, B, Hq, Hkv, N, D, Bq, Bk, causal, stream) -> int:
+    return load().bsfa_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(tau), _ptr(out), _ptr(lse), _ptr(block_mask),
+                               B, Hq, Hkv, N, D, Bq, Bk, int(bool(causal)), _stream(stream))
+
+
+def bsfa_validate(B, Hq, Hkv, N, D, Bq, Bk, causal) -> int:
+    return load().bsfa_validate(B, Hq, Hkv, N, D, Bq, Bk, int(bool(causal)))
+
+
+def bsfa_get_status(stream=None) -> int:
+    return load().bsfa_get_status(_stream(stream))
+
+
+def bsfa_status_string(status: int) -> str:
+    return load().bsfa_status_string(status).decode()
+
+
+def bsfa_last_error() -> str:
+    return load().bsfa_last_error().decode()
+
+
+# ----------------------------------------------------------------------------- torch conveniences
+
+def _check(status: int):
+    if status != BSFA_OK:
+        raise BsfaError(status, bsfa_last_error())
+
+
+def forward(q, k, v, tau, *, Bq: int, Bk: int, causal: bool, want_lse: bool = True, want_mask: bool = False,
+            out=None, lse=None, block_mask=None, stream=None):
+    """Run the forward on device tensors. q: bf16 [B,N,Hq,D]; k, v: bf16 [B,N,Hkv,D]; tau: fp32 [Hq].
+
+    Returns (out, lse or None, block_mask or None). Outputs are allocated with torch
+    unless given.
+    """
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or t.dim() != 4:
+            raise ValueError(f"{name} must be a contiguous 4-D bf16 CUDA tensor")
+    if tau.dtype != torch.float32 or not tau.is_cuda or tau.numel() != q.shape[2]:
+        raise ValueError("tau must be a float32 CUDA tensor with one value per query head")
+    B, N, Hq, D = q.shape
+    Hkv = k.shape[2]
+    if k.shape != (B, N, Hkv, D) or v.shape != k.shape:
+        raise ValueError("k and v must be [B, N, Hkv, D] with q's B, N and D")
+    if out is None:
+        out = torch.empty_like(q)
+    if want_lse and lse is None:
+        lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
+    if want_mask and block_mask is None:
+        block_mask = torch.empty((B, Hq, N // Bq, N // Bk), dtype=torch.uint8, device=q.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    _check(bsfa_forward(q, k, v, tau, out, lse if want_lse else None, block_mask if want_mask else None,
+                        B, Hq, Hkv, N, D, Bq, Bk, causal, stream))
+    return out, (lse if want_lse else None), (block_mask if want_mask else None)
+
+
+def forward_host(q, k, v, tau, *, Bq: int, Bk: int, causal: bool, device=None, stream=None, bufs=None):
+    """End-to-end call on host tensors: copy inputs to the device, run, copy out and lse back.
+
+    q, k, v: bf16 CPU tensors (pinned for asynchronous copies); tau: fp32 CPU tensor.
+    ``bufs`` (from ``device_buffers``) holds reusable device and pinned host buffers.
+    Returns (out_host, lse_host).
+    """
+    import torch
+    device = torch.device("cuda") if device is None else device
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    if bufs is None:
+        bufs = device_buffers(q.shape, k.shape, device)
+    with torch.cuda.stream(stream):
+        for name, src in (("q", q), ("k", k), ("v", v), ("tau", tau)):
+            bufs[name].copy_(src, non_blocking=True)
+        forward(bufs["q"], bufs["k"], bufs["v"], bufs["tau"], Bq=Bq, Bk=Bk, causal=causal, out=bufs["out"],
+                lse=bufs["lse"], stream=stream)
+        bufs["out_host"].copy_(bufs["out"], non_blocking=True)
+        bufs["lse_host"].copy_(bufs["lse"], non_blocking=True)
+    stream.synchronize()
+    return bufs["out_host"], bufs["lse_host"]
+
+
+def device_buffers(q_shape, kv_shape, device):
+    """Device inputs/outputs plus pinned host outputs for ``forward_host``."""
+    import torch
+    B, N, Hq, D = q_shape
+    return {
+        "q": torch.empty(q_shape, dtype=torch.bfloat16, device=device),
+        "k": torch.empty(kv_shape, dtype=torch.bfloat16, device=device),
+        "v": torch.empty(kv_shape, dtype=torch.bfloat16, device=device),
+        "tau": torch.empty((Hq,), dtype=torch.float32, device=device),
+        "out": torch.empty(q_shape, dtype=torch.bfloat16, device=device),
+        "lse": torch.empty((B, Hq, N), dtype=torch.float32, device=device),
+        "out_host": torch.empty(q_shape, dtype=torch.bfloat16, pin_memory=True),
+        "lse_host": torch.empty((B, Hq, N), dtype=torch.float32, pin_memory=True),
+    }

@@ -1,0 +1,193 @@
+// C ABI of the BSFA prefill forward: argument validation, TMA descriptor
+// encoding, kernel dispatch and the device status word. The declarations and
+// their contracts are in include/bsfa.h.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include "bsfa.h"
+#include "bsfa_launch.cuh"
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+bsfa_status fail(bsfa_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+bsfa_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(BSFA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// One status word per device: kernels OR a nonzero value into it when they give
+// up on a bounded wait.
+__device__ int g_status_word;
+
+constexpr int kMaxDevices = 64;
+std::mutex g_dev_mutex;
+int* g_status_ptr[kMaxDevices] = {};
+int g_cc_major[kMaxDevices] = {};
+
+bsfa_status device_setup(int dev, int** status_ptr) {
+  if (dev < 0 || dev >= kMaxDevices) return fail(BSFA_ERR_UNSUPPORTED, "device index %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_dev_mutex);
+  if (g_status_ptr[dev] == nullptr) {
+    int major = 0;
+    cudaError_t e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    g_cc_major[dev] = major;
+    if (major != 10) return fail(BSFA_ERR_UNSUPPORTED, "device %d has compute capability %d.x; sm_100 required", dev, major);
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_status_word);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(status word)");
+    g_status_ptr[dev] = static_cast<int*>(p);
+  }
+  if (g_cc_major[dev] != 10) return fail(BSFA_ERR_UNSUPPORTED, "device %d is not sm_100", dev);
+  *status_ptr = g_status_ptr[dev];
+  return BSFA_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// [B, N, H, D] bf16, boxes of 64 (D) x 1 (head) x rows (N) x 1 (batch), 128-byte swizzle.
+bool encode_bnhd(CUtensorMap* map, const void* ptr, int B, int N, int H, int D, int rows) {
+  auto encode = tensor_map_encoder();
+  if (encode == nullptr) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)N, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)N * H * D * 2};
+  cuuint32_t box[4] = {64, 1, (cuuint32_t)rows, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+}  // namespace
+
+extern "C" {
+
+bsfa_status bsfa_validate(int B, int Hq, int Hkv, int N, int D, int Bq, int Bk, int causal) {
+  (void)causal;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || N <= 0 || D <= 0 || Bq <= 0 || Bk <= 0)
+    return fail(BSFA_ERR_INVALID_ARG, "sizes must be positive (B=%d Hq=%d Hkv=%d N=%d D=%d Bq=%d Bk=%d)", B, Hq, Hkv,
+                N, D, Bq, Bk);
+  if (Hq % Hkv != 0) return fail(BSFA_ERR_INVALID_ARG, "Hq=%d is not a multiple of Hkv=%d", Hq, Hkv);
+  if (D != 64 && D != 128) return fail(BSFA_ERR_UNSUPPORTED, "D=%d unsupported (64 or 128)", D);
+  if ((Bq != 64 && Bq != 128) || (Bk != 64 && Bk != 128))
+    return fail(BSFA_ERR_UNSUPPORTED, "Bq=%d, Bk=%d unsupported (64 or 128)", Bq, Bk);
+  if (N % 128 != 0) return fail(BSFA_ERR_UNSUPPORTED, "N=%d must be a multiple of 128", N);
+  const long long rows = (long long)B * N, head_rows = (long long)B * Hq * N;
+  if (rows > 0x7fffffffLL || head_rows > 0x7fffffffLL)
+    return fail(BSFA_ERR_UNSUPPORTED, "B*Hq*N=%lld exceeds the 32-bit row index", head_rows);
+  return BSFA_OK;
+}
+
+bsfa_status bsfa_forward(const void* q, const void* k, const void* v, const float* tau, void* out, float* lse,
+                         uint8_t* block_mask, int B, int Hq, int Hkv, int N, int D, int Bq, int Bk, int causal,
+                         void* stream) {
+  bsfa_status st = bsfa_validate(B, Hq, Hkv, N, D, Bq, Bk, causal);
+  if (st != BSFA_OK) return st;
+  if (!q || !k || !v || !tau || !out) return fail(BSFA_ERR_INVALID_ARG, "q, k, v, tau and out must be non-null");
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16))
+    return fail(BSFA_ERR_INVALID_ARG, "q, k, v and out must be 16-byte aligned");
+  if (!aligned(tau, 4) || (lse && !aligned(lse, 4))) return fail(BSFA_ERR_INVALID_ARG, "tau and lse must be 4-byte aligned");
+
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  int* status_ptr = nullptr;
+  st = device_setup(dev, &status_ptr);
+  if (st != BSFA_OK) return st;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (block_mask) {
+    const size_t n = (size_t)B * Hq * (size_t)(N / Bq) * (size_t)(N / Bk);
+    e = cudaMemsetAsync(block_mask, 3, n, s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(block_mask)");
+  }
+
+  CUtensorMap tq, tk, tv;
+  if (!encode_bnhd(&tq, q, B, N, Hq, D, 128) || !encode_bnhd(&tk, k, B, N, Hkv, D, Bk) ||
+      !encode_bnhd(&tv, v, B, N, Hkv, D, Bk))
+    return fail(BSFA_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+
+  bsfa::FwdParams p;
+  p.tau = tau;
+  p.out = static_cast<uint16_t*>(out);
+  p.lse = lse;
+  p.mask = block_mask;
+  p.status = status_ptr;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.N = N;
+  p.group = Hq / Hkv;
+  p.scale = (float)(1.0 / std::sqrt((double)D));
+  p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
+  const int grid = B * Hq * (N / 128);
+  e = (D == 64) ? bsfa::launch_fwd_d64(tq, tk, tv, p, Bq, Bk, causal != 0, block_mask != nullptr, grid, s)
+                : bsfa::launch_fwd_d128(tq, tk, tv, p, Bq, Bk, causal != 0, block_mask != nullptr, grid, s);
+  if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+  return BSFA_OK;
+}
+
+bsfa_status bsfa_get_status(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  int dev = 0;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  int* status_ptr = nullptr;
+  bsfa_status st = device_setup(dev, &status_ptr);
+  if (st != BSFA_OK) return st;
+  int word = 0;
+  e = cudaMemcpy(&word, status_ptr, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(status word)");
+  if (word != 0) {
+    const int zero = 0;
+    e = cudaMemcpy(status_ptr, &zero, sizeof(int), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(clear status word)");
+    return fail(BSFA_ERR_DEVICE_TIMEOUT, "a kernel gave up on a bounded wait (status word 0x%x)", word);
+  }
+  return BSFA_OK;
+}
+
+const char* bsfa_status_string(bsfa_status s) {
+  switch (s) {
+    case BSFA_OK: return "BSFA_OK";
+    case BSFA_ERR_INVALID_ARG: return "BSFA_ERR_INVALID_ARG";
+    case BSFA_ERR_UNSUPPORTED: return "BSFA_ERR_UNSUPPORTED";
+    case BSFA_ERR_CUDA: return "BSFA_ERR_CUDA";
+    case BSFA_ERR_DEVICE_TIMEOUT: return "BSFA_ERR_DEVICE_TIMEOUT";
+  }
+  return "BSFA_UNKNOWN_STATUS";
+}
+
+const char* bsfa_last_error(void) { return g_last_error; }
+
+}  // extern "C"

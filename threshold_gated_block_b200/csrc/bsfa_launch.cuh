@@ -1,0 +1,46 @@
+// Kernel instantiation and launch for one head dimension (used by the per-D
+// translation units so the 32 kernel variants compile in parallel).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "bsfa_fwd_kernel.cuh"
+
+namespace bsfa {
+
+template <int D, int BQ, int BK, bool CAUSAL, bool MASK>
+cudaError_t launch_variant(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
+                           int grid, cudaStream_t stream) {
+  using S = FwdShape<D, BQ, BK>;
+  auto kern = bsfa_fwd_kernel<D, BQ, BK, CAUSAL, MASK>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kThreads, S::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
+                       int Bq, int Bk, bool causal, bool mask, int grid, cudaStream_t s) {
+#define BSFA_CASE(BQ, BK)                                                                          \
+  if (Bq == BQ && Bk == BK) {                                                                      \
+    if (causal)                                                                                    \
+      return mask ? launch_variant<D, BQ, BK, true, true>(tq, tk, tv, p, grid, s)                  \
+                  : launch_variant<D, BQ, BK, true, false>(tq, tk, tv, p, grid, s);                \
+    return mask ? launch_variant<D, BQ, BK, false, true>(tq, tk, tv, p, grid, s)                   \
+                : launch_variant<D, BQ, BK, false, false>(tq, tk, tv, p, grid, s);                 \
+  }
+  BSFA_CASE(64, 64)
+  BSFA_CASE(64, 128)
+  BSFA_CASE(128, 64)
+  BSFA_CASE(128, 128)
+#undef BSFA_CASE
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_fwd_d64(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const FwdParams&, int, int,
+                           bool, bool, int, cudaStream_t);
+cudaError_t launch_fwd_d128(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const FwdParams&, int, int,
+                            bool, bool, int, cudaStream_t);
+
+}  // namespace bsfa
