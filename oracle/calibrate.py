@@ -8,10 +8,10 @@ blocks, averaged over calibration samples ("Block Sparse Flash Attention",
 The workloads here use one threshold per query head, so the same rule is taken
 per head over every gated (visible, off-diagonal) block of that head: sort the
 block maxima ascending, and for a target skip fraction p put tau in the gap
-between the n-th and (n+1)-th values, n = round(p * count). tau is the midpoint
-of that gap, rounded to float32. When the gap is narrower than ``min_gap`` the
-nearest wider gap is used instead, so no block maximum sits within rounding of
-tau. The achieved skip fraction is reported, not assumed.
+near the n-th value, n = round(p * count): among the ranks within 0.2% of n it
+takes the widest gap between neighbouring maxima and puts tau at its midpoint,
+rounded to float32, so that tau sits as far as it can from every block maximum.
+The achieved skip fraction is reported, not assumed.
 """
 from __future__ import annotations
 
@@ -19,11 +19,18 @@ import numpy as np
 
 from .bsfa_oracle import CODE_SKIPPED, block_maxima
 
-MIN_GAP = 4e-4
+RANK_WINDOW = 0.002
 
 
-def tau_for_skip(values: np.ndarray, p: float, min_gap: float = MIN_GAP) -> float:
-    """Threshold that skips a fraction ~p of ``values`` (block maxima), as a float32 value."""
+def tau_for_skip(values: np.ndarray, p: float, window: float = RANK_WINDOW) -> float:
+    """Threshold that skips a fraction ~p of ``values`` (block maxima), as a float32 value.
+
+    With the values sorted ascending and n = round(p * count), tau is the midpoint
+    of the widest gap a[m-1] < tau <= a[m] among the ranks m within
+    +-round(window * count) of n (ties go to the rank nearest n). This keeps the
+    skipped fraction within ``window`` of p while keeping tau as far as possible
+    from every block maximum.
+    """
     a = np.sort(np.asarray(values, dtype=np.float64))
     n_total = len(a)
     if n_total == 0:
@@ -33,14 +40,13 @@ def tau_for_skip(values: np.ndarray, p: float, min_gap: float = MIN_GAP) -> floa
         return float(np.float32(a[0] - 1.0))
     if n >= n_total:
         return float(np.float32(a[-1] + 1.0))
-    # Candidate gaps a[m-1] < tau <= a[m], nearest to n first.
-    order = sorted(range(1, n_total), key=lambda m: (abs(m - n), m))
+    w = int(round(window * n_total))
+    ranks = range(max(1, n - w), min(n_total - 1, n + w) + 1)
+    order = sorted(ranks, key=lambda m: (-(a[m] - a[m - 1]), abs(m - n), m))
     for m in order:
-        lo, hi = a[m - 1], a[m]
-        if hi - lo >= min_gap:
-            t = np.float32(0.5 * (lo + hi))
-            if lo < float(t) < hi and float(t) - lo >= min_gap / 4 and hi - float(t) >= min_gap / 4:
-                return float(t)
+        t = float(np.float32(0.5 * (a[m - 1] + a[m])))
+        if a[m - 1] < t <= a[m]:
+            return t
     return float(np.float32(0.5 * (a[n - 1] + a[n])))
 
 
