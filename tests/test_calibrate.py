@@ -15,9 +15,18 @@ def test_tau_sits_in_the_gap_at_the_target_rank():
     assert tau_for_skip([1.0, 2.0, 3.0, 4.0], 0.25) == 1.5
 
 
-def test_narrow_gaps_are_avoided():
+def test_widest_gap_within_the_rank_window():
+    # 2000 maxima 1e-5 apart with one 1e-3 gap two ranks above the target rank
+    a = np.cumsum(np.full(2000, 1e-5)) + 3.0
+    a[1002:] += 1e-3
+    t = tau_for_skip(a, 0.5)                 # window = round(0.002 * 2000) = 4 ranks
+    assert a[1001] < t < a[1002]
+    assert (a < t).sum() == 1002
+
+
+def test_small_counts_cut_at_the_exact_rank():
     t = tau_for_skip([1.0, 1.0001, 2.0, 3.0], 0.25)
-    assert 1.0001 < t < 2.0
+    assert 1.0 < t < 1.0001
 
 
 def test_extreme_fractions():
