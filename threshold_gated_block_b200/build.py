@@ -8,6 +8,7 @@ from __future__ import annotations
 
 import concurrent.futures as cf
 import os
+import re
 import shutil
 import subprocess
 import sys
@@ -21,13 +22,34 @@ LIB = os.path.join(PKG, "libbsfa.so")
 SOURCES = ["bsfa_api.cu", "bsfa_fwd_d64.cu", "bsfa_fwd_d128.cu"]
 HEADERS = ["ptx.cuh", "bsfa_fwd_kernel.cuh", "bsfa_launch.cuh"]
 
+# The forward kernel re-balances registers between its warpgroups
+# (setmaxnreg); the split is sized for exactly this launch budget per thread, so
+# the build refuses a kernel compiled with any other count.
+FWD_KERNEL_REGS = 168
+
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-O3", "-std=c++17", "-lineinfo",
     "-Xcompiler", "-fPIC",
     "--expt-relaxed-constexpr",
     "-I", INCLUDE, "-I", CSRC,
+    "-Xptxas", "-v",
 ]
+
+
+def check_registers(ptxas_log: str) -> None:
+    """Every bsfa_fwd_kernel variant must be compiled with FWD_KERNEL_REGS registers."""
+    entry = None
+    for line in ptxas_log.splitlines():
+        m = re.search(r"Compiling entry function '([^']+)'", line)
+        if m:
+            entry = m.group(1)
+            continue
+        m = re.search(r"Used (\d+) registers", line)
+        if m and entry and "bsfa_fwd_kernel" in entry:
+            if int(m.group(1)) != FWD_KERNEL_REGS:
+                raise RuntimeError(f"{entry}: {m.group(1)} registers, expected {FWD_KERNEL_REGS}")
+            entry = None
 
 
 def nvcc() -> str:
@@ -63,6 +85,7 @@ def build(force: bool = False, verbose: bool = False, extra_flags: list[str] | N
             raise RuntimeError(f"nvcc failed: {' '.join(cmd)}\n{r.stdout}\n{r.stderr}")
         if verbose and (r.stdout or r.stderr):
             print(r.stdout, r.stderr, file=sys.stderr)
+        check_registers(r.stdout + r.stderr)
         return r
 
     with cf.ThreadPoolExecutor(max_workers=len(jobs) or 1) as ex:
@@ -74,5 +97,4 @@ def build(force: bool = False, verbose: bool = False, extra_flags: list[str] | N
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose=True,
-                extra_flags=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else None))
+    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv))

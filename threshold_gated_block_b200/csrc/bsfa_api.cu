@@ -147,9 +147,13 @@ bsfa_status bsfa_forward(const void* q, const void* k, const void* v, const floa
   p.Hkv = Hkv;
   p.N = N;
   p.group = Hq / Hkv;
+  // A CTA pairs two query heads of one KV group when the group size is even,
+  // otherwise two adjacent 128-row tiles of one head.
+  p.pair_heads = (p.group % 2 == 0) ? 1 : 0;
   p.scale = (float)(1.0 / std::sqrt((double)D));
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
-  const int grid = B * Hq * (N / 128);
+  const int tiles = N / 128;
+  const int grid = p.pair_heads ? B * (Hq / 2) * tiles : B * Hq * ((tiles + 1) / 2);
   e = (D == 64) ? bsfa::launch_fwd_d64(tq, tk, tv, p, Bq, Bk, causal != 0, block_mask != nullptr, grid, s)
                 : bsfa::launch_fwd_d128(tq, tk, tv, p, Bq, Bk, causal != 0, block_mask != nullptr, grid, s);
   if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
