@@ -395,7 +395,8 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, Bars* bars, uin
     __syncwarp();
     if (!keep_any) {                 // skipped by every tile of the slot: release S, nothing else
       tc_fence_before();
-      mbar_arrive(&bars->p_full[s]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->p_full[s]);
       continue;
     }
 
@@ -414,27 +415,32 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, Bars* bars, uin
       }
       l *= alpha;
     }
+    // P = 2^(s * log2(e)/sqrt(d) - m): half of the exponentials on the SFU (ex2),
+    // half as a polynomial on the FMA pipe, all other arithmetic in f32x2 pairs.
     const bool live = my_keep && (m != -INFINITY);
-    const float neg_m = live ? -m : 0.f;
-    float ls0 = 0.f, ls1 = 0.f, ls2 = 0.f, ls3 = 0.f;
+    const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
+    const float2 nm2 = make_float2(-m, -m);
+    float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
     uint32_t pk[BK / 2];
 #pragma unroll
     for (int e = 0; e < BK / 2; e += 2) {
-      float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
-      if (live) {
-        p0 = ex2_approx(fmaf(sv[2 * e], p.scale_log2, neg_m));
-        p1 = ex2_approx(fmaf(sv[2 * e + 1], p.scale_log2, neg_m));
-        p2 = ex2_approx(fmaf(sv[2 * e + 2], p.scale_log2, neg_m));
-        p3 = ex2_approx(fmaf(sv[2 * e + 3], p.scale_log2, neg_m));
-      }
-      ls0 += p0;
-      ls1 += p1;
-      ls2 += p2;
-      ls3 += p3;
-      pk[e] = pack_bf16x2(p0, p1);
-      pk[e + 1] = pack_bf16x2(p2, p3);
+      const float2 xa = __ffma2_rn(make_float2(sv[2 * e], sv[2 * e + 1]), sl2, nm2);
+      const float2 xb = __ffma2_rn(make_float2(sv[2 * e + 2], sv[2 * e + 3]), sl2, nm2);
+      const float2 pa = make_float2(ex2_approx(xa.x), ex2_approx(xa.y));
+      const float2 pb = exp2_poly2(xb);
+      acc0 = __fadd2_rn(acc0, pa);
+      acc1 = __fadd2_rn(acc1, pb);
+      pk[e] = pack_bf16x2(pa.x, pa.y);
+      pk[e + 1] = pack_bf16x2(pb.x, pb.y);
     }
-    l += (ls0 + ls1) + (ls2 + ls3);
+    if (__any_sync(0xffffffffu, !live)) {   // rows this block does not update: P = 0
+      if (!live) {
+#pragma unroll
+        for (int e = 0; e < BK / 2; ++e) pk[e] = 0u;
+        acc0 = acc1 = make_float2(0.f, 0.f);
+      }
+    }
+    l += (acc0.x + acc0.y) + (acc1.x + acc1.y);
     if constexpr (BK == 128) tmem_st_x64(s_tmem, pk);   // P (bf16 pairs) over the consumed S columns
     else tmem_st_x32(s_tmem, pk);
     tmem_st_wait();
@@ -452,7 +458,8 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, Bars* bars, uin
       tmem_st_wait();
     }
     tc_fence_before();
-    mbar_arrive(&bars->p_full[s]);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bars->p_full[s]);
   }
 
   // Epilogue: O / l -> bf16 rows, lse = ln-sum-exp over the kept set.
@@ -500,7 +507,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < S::VS; ++i) { mbar_init(&bars->v_full[i], 1); mbar_init(&bars->v_empty[i], 1); }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars->s_full[i], 1);
-      mbar_init(&bars->p_full[i], 128);
+      mbar_init(&bars->p_full[i], 4);          // one arrival per softmax warp
       mbar_init(&bars->o_done[i], 1);
       for (int g = 0; g < S::GR; ++g) { mbar_init(&bars->gate_full[i][g], 1); mbar_init(&bars->gate_empty[i][g], 1); }
     }

@@ -303,6 +303,26 @@ __device__ __forceinline__ float warp_max_redux(float v) {
   return d;
 }
 
+// 2^x for x <= 8 on the FMA pipe, two lanes at a time: x = i + f with i = round(x)
+// and f in [-1/2, 1/2]; 2^f is the degree-3 minimax polynomial of
+// fit_exp2_poly.py (max relative error 7.5e-5) and 2^i is added to the
+// exponent field. x is clamped at -125.5 so the result stays a normal float
+// (>= 2^-126), which is zero for every purpose of the softmax.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kRound = 12582912.f;   // 1.5 * 2^23: x + kRound holds round(x) in its low mantissa bits
+  constexpr float kC0 = 0.99992806f, kC1 = 0.69326097f, kC2 = 0.24261113f, kC3 = 0.05517167f;
+  x.x = fmaxf(x.x, -125.5f);
+  x.y = fmaxf(x.y, -125.5f);
+  const float2 t = __fadd2_rn(x, make_float2(kRound, kRound));
+  const float2 r = __fadd2_rn(t, make_float2(-kRound, -kRound));
+  const float2 f = __ffma2_rn(r, make_float2(-1.f, -1.f), x);
+  float2 q = __ffma2_rn(make_float2(kC3, kC3), f, make_float2(kC2, kC2));
+  q = __ffma2_rn(q, f, make_float2(kC1, kC1));
+  q = __ffma2_rn(q, f, make_float2(kC0, kC0));
+  return make_float2(__int_as_float(__float_as_int(t.x) * (1 << 23) + __float_as_int(q.x)),
+                     __int_as_float(__float_as_int(t.y) * (1 << 23) + __float_as_int(q.y)));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
