@@ -61,8 +61,8 @@ typedef enum {
  *   causal     nonzero for causal prefill, zero for bidirectional attention
  *   stream     a cudaStream_t (NULL = the legacy default stream)
  *
- * Supported: D in {64, 128}; Bq, Bk in {64, 128}; N a positive multiple of 128;
- * an sm_100 device. The caller owns every buffer; results are valid once the
+ * Supported: D in {64, 128}; Bq, Bk in {64, 128}; N a positive multiple of 128
+ * with at most 4096 key blocks (N / Bk <= 4096); an sm_100 device. The caller owns every buffer; results are valid once the
  * stream has reached the call. Returns BSFA_OK once the kernel is enqueued;
  * argument errors are returned before any CUDA call is made. A kernel that gives
  * up on a bounded internal wait leaves `out` undefined and sets the device

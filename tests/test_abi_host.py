@@ -53,6 +53,8 @@ def test_status_strings(lib):
     ((1, 32, 8, 8192, 128, 128, 256, 1), bsfa.BSFA_ERR_UNSUPPORTED),
     ((1, 32, 8, 8000, 128, 128, 128, 1), bsfa.BSFA_ERR_UNSUPPORTED),
     ((1024, 64, 8, 65536, 128, 128, 128, 1), bsfa.BSFA_ERR_UNSUPPORTED),
+    ((1, 8, 8, 4096 * 64, 64, 64, 64, 1), bsfa.BSFA_OK),
+    ((1, 8, 8, 4096 * 64 + 128, 64, 64, 64, 1), bsfa.BSFA_ERR_UNSUPPORTED),
 ])
 def test_validate(lib, args, want):
     assert bsfa.bsfa_validate(*args) == want

@@ -101,6 +101,8 @@ bsfa_status bsfa_validate(int B, int Hq, int Hkv, int N, int D, int Bq, int Bk, 
   if ((Bq != 64 && Bq != 128) || (Bk != 64 && Bk != 128))
     return fail(BSFA_ERR_UNSUPPORTED, "Bq=%d, Bk=%d unsupported (64 or 128)", Bq, Bk);
   if (N % 128 != 0) return fail(BSFA_ERR_UNSUPPORTED, "N=%d must be a multiple of 128", N);
+  if (N / Bk > bsfa::kMaxKeyBlocks)
+    return fail(BSFA_ERR_UNSUPPORTED, "N/Bk=%d exceeds %d key blocks", N / Bk, bsfa::kMaxKeyBlocks);
   const long long rows = (long long)B * N, head_rows = (long long)B * Hq * N;
   if (rows > 0x7fffffffLL || head_rows > 0x7fffffffLL)
     return fail(BSFA_ERR_UNSUPPORTED, "B*Hq*N=%lld exceeds the 32-bit row index", head_rows);

@@ -50,28 +50,30 @@ struct FwdParams {
 // exp2 domain; until then P is taken against the stale maximum (values <= 2^8,
 // exact in the final O / l ratio).
 constexpr float kRescaleThreshold = 8.0f;
-constexpr int kThreads = 384;
-constexpr int kLaunchRegs = 168;      // 65536 / 384, rounded down to the allocation granularity
-constexpr int kSoftmaxRegs = 216;
-constexpr int kProducerRegs = 72;
-static_assert(2 * 128 * kSoftmaxRegs + 128 * kProducerRegs <= kThreads * kLaunchRegs, "register split");
+// Threads that share one query row in the softmax (each holds Bk/kRowSplit key columns).
+constexpr int kRowSplit = 2;
+constexpr int kSoftmaxWarps = 4 * kRowSplit;
+constexpr int kThreads = 32 * (kSoftmaxWarps + 4);
+constexpr int kLaunchRegs = kRowSplit == 2 ? 168 : 96;   // 65536 / kThreads, rounded down to the allocation granularity
+constexpr int kSoftmaxRegs = kRowSplit == 2 ? 216 : 104;
+constexpr int kProducerRegs = kRowSplit == 2 ? 72 : 64;
+static_assert(kSoftmaxWarps * 32 * kSoftmaxRegs + 128 * kProducerRegs <= kThreads * kLaunchRegs, "register split");
 
 template <int D, int BQ, int BK>
 struct FwdShape {
   static constexpr int ROWS = 128;
   static constexpr int NSUB = ROWS / BQ;   // query tiles per slot
   static constexpr int DCH = D / 64;       // 128-byte swizzle chunks along D
-  static constexpr int KS = 3;             // K ring depth
+  static constexpr int KS = 2;             // K ring depth
   static constexpr int VS = 2;             // V ring depth
-  static constexpr int GR = 4;             // gate-decision ring depth (per slot)
   static constexpr uint32_t Q_BYTES = ROWS * D * 2;
   static constexpr uint32_t KV_BYTES = BK * D * 2;
   static constexpr uint32_t OFF_Q = 0;                        // two Q tiles
   static constexpr uint32_t OFF_K = OFF_Q + 2 * Q_BYTES;
   static constexpr uint32_t OFF_V = OFF_K + KS * KV_BYTES;
   static constexpr uint32_t OFF_BAR = OFF_V + VS * KV_BYTES;
-  static constexpr uint32_t BAR_BYTES = 1024;
-  static constexpr uint32_t SMEM_BYTES = OFF_BAR + BAR_BYTES + 1024;   // + alignment slack
+  static constexpr uint32_t BAR_BYTES = 6144;                       // barriers, gate bits, softmax exchange
+  static constexpr uint32_t SMEM_BYTES = OFF_BAR + BAR_BYTES;        // base is 1024-aligned (checked)
   static constexpr uint32_t TMEM_S0 = 0;
   static constexpr uint32_t TMEM_O0 = 2 * BK;
   static constexpr uint32_t TMEM_COLS = (2 * BK + 2 * D <= 256) ? 256 : 512;
@@ -81,19 +83,23 @@ struct FwdShape {
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
 
-template <int KS, int VS, int GR>
+// Gate decisions of every block, one bit per (slot, block): at most this many
+// key blocks per sequence.
+constexpr int kMaxKeyBlocks = 4096;
+
+template <int KS, int VS>
 struct alignas(8) FwdBarriers {
   uint64_t q_full;
   uint64_t k_full[KS], k_empty[KS];
   uint64_t v_full[VS], v_empty[VS];
   uint64_t s_full[2], p_full[2], o_done[2];
-  uint64_t gate_full[2][GR], gate_empty[2][GR];
   uint64_t drain;
   uint32_t tmem_base;
-  int abort;
-  int gate_flag[2][GR];
-  int p_keep[2];
-  float red[2][2][4];   // [slot][block parity][warp]
+  int abort;                               // any role gave up on a bounded wait
+  int sm_abort[2];                         // softmax warps' agreement to stop, by block parity
+  int decided[2];                          // blocks whose gate decision is published, per slot
+  uint32_t gate_bits[2][kMaxKeyBlocks / 32];
+  float xch[2 * kRowSplit * 128];          // partial row maxima [slot][part][row]; normalisers [part][row] at the end
 };
 
 struct FwdUnit {
@@ -175,26 +181,42 @@ __device__ __forceinline__ void kq_producer(const CUtensorMap* tm_q, const CUten
     drain_wait(&bars->k_full[t % S::KS], (t / S::KS) & 1);
 }
 
-// ---------------------------------------------------------------------------- V producer (warp 10, one thread)
+// Bounded spin until slot s's gate decision for block j is published.
+template <typename Bars>
+__device__ __forceinline__ bool wait_decided(Bars* bars, int s, int j) {
+  volatile int* decided = &bars->decided[s];
+  volatile int* abort_flag = &bars->abort;
+  if (*decided > j) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (;;) {
+#pragma unroll 1
+    for (int i = 0; i < 256; ++i)
+      if (*decided > j) return true;
+    if (*abort_flag) return false;
+    if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+      *abort_flag = 1;
+      return false;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------- V producer (one thread)
 
 template <int D, int BQ, int BK, typename Bars>
 __device__ __forceinline__ void v_producer(const CUtensorMap* tm_v, uint8_t* smem, Bars* bars, const FwdUnit& w) {
   using S = FwdShape<D, BQ, BK>;
   volatile int* abort_flag = &bars->abort;
-  volatile int* gate_flag = &bars->gate_flag[0][0];
   prefetch_tensormap(tm_v);
   const int nblk = max(w.nblk[0], w.nblk[1]);
   int v_count = 0;
   bool failed = false;
   for (int j = 0; j < nblk && !failed; ++j) {
-    const int g = j % S::GR;
     bool loaded = false;
 #pragma unroll
     for (int s = 0; s < 2; ++s) {
       if (j >= w.nblk[s]) continue;
-      if (!mbar_wait(&bars->gate_full[s][g], (j / S::GR) & 1, abort_flag)) { failed = true; break; }
-      const int keep = gate_flag[s * S::GR + g];
-      mbar_arrive(&bars->gate_empty[s][g]);
+      if (!wait_decided(bars, s, j)) { failed = true; break; }
+      const bool keep = (((volatile uint32_t*)bars->gate_bits[s])[j >> 5] >> (j & 31)) & 1u;
       if (!keep || loaded) continue;     // skipped by this slot (or already requested)
       const int slot = v_count % S::VS;
       if (!mbar_wait(&bars->v_empty[slot], ((v_count / S::VS) & 1) ^ 1, abort_flag)) { failed = true; break; }
@@ -219,7 +241,8 @@ __device__ __forceinline__ void mma_issuer(uint8_t* smem, Bars* bars, uint32_t t
   constexpr uint32_t IDESC_QK = make_idesc_bf16(128, BK, false);   // B = K tile, K-major
   constexpr uint32_t IDESC_PV = make_idesc_bf16(128, D, true);     // B = V tile, MN-major
   volatile int* abort_flag = &bars->abort;
-  volatile int* p_keep = bars->p_keep;
+  volatile uint32_t* bits0 = bars->gate_bits[0];
+  volatile uint32_t* bits1 = bars->gate_bits[1];
   const int nblk = max(w.nblk[0], w.nblk[1]);
 
   auto qk = [&](int s, int kslot) {
@@ -267,7 +290,8 @@ __device__ __forceinline__ void mma_issuer(uint8_t* smem, Bars* bars, uint32_t t
         if (j >= w.nblk[s]) continue;
         if (!mbar_wait(&bars->p_full[s], j & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        if (p_keep[s]) {
+        const uint32_t word = s ? bits1[j >> 5] : bits0[j >> 5];
+        if ((word >> (j & 31)) & 1u) {
           if (!v_ready) {
             vslot = v_count % S::VS;
             if (!mbar_wait(&bars->v_full[vslot], (v_count / S::VS) & 1, abort_flag)) { ok = false; break; }
@@ -301,188 +325,256 @@ __device__ __forceinline__ void mma_issuer(uint8_t* smem, Bars* bars, uint32_t t
   drain_wait(&bars->drain, 0);
 }
 
-// ---------------------------------------------------------------------------- softmax / gate / epilogue (warps 0-7)
+// ---------------------------------------------------------------------------- softmax / gate / epilogue (warps 0-15)
 
+// All softmax warps work on one slot at a time and alternate between the two
+// slots block by block, so a slot's softmax always overlaps the other slot's
+// MMAs. Warp w reads TMEM lanes 32*(w%4)..+31 (its rows) and key columns
+// [(w/4)*Bk/R, (w/4+1)*Bk/R), R = kRowSplit threads sharing each row. Partial row maxima
+// cross warps through shared memory; the gate decision itself is the OR that
+// the block's named barrier computes over the threads' own comparisons.
+template <int BK>
+struct SoftmaxRow {
+  float m[2] = {-INFINITY, -INFINITY};   // running row maximum per slot, exp2 domain
+  float l[2] = {0.f, 0.f};               // this thread's share of the running normaliser per slot
+};
+
+// Returns 2 when every softmax thread agreed to abort (a bounded wait gave up
+// somewhere), otherwise this thread's own failure flag (0 or 1), which the next
+// barrier folds into that agreement.
 template <int D, int BQ, int BK, bool CAUSAL, bool WRITE_MASK, typename Bars>
-__device__ __forceinline__ void softmax_role(const FwdParams& p, Bars* bars, uint32_t tmem, const FwdUnit& w) {
+__device__ __forceinline__ int softmax_block(const FwdParams& p, Bars* bars, uint32_t tmem, const FwdUnit& w,
+                                             int s, int j, float tau, SoftmaxRow<BK>& st, bool failed) {
   using S = FwdShape<D, BQ, BK>;
+  constexpr int QC = BK / kRowSplit;         // key columns per thread
+  constexpr int QD = D / kRowSplit;          // output columns per thread
   volatile int* abort_flag = &bars->abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int s = warp >> 2;                 // slot
-  const int wid = warp & 3;                // warp within the slot's warpgroup
-  const int r = wid * 32 + lane;           // row within the slot, TMEM lane
-  // (selects rather than runtime indexing keep the unit in registers)
-  const int nblk = s ? w.nblk[1] : w.nblk[0];
-  if (nblk == 0) return;                   // slot past the end of the sequence
+  const int c4 = warp >> 2;                  // column part
+  const int q = warp & 3;                    // TMEM lane quarter
+  const int r = q * 32 + lane;               // row within the slot, TMEM lane
   const int hq = s ? w.hq[1] : w.hq[0];
   const int q0 = s ? w.q0[1] : w.q0[0];
-  const int b = w.b;
   const int qrow = q0 + r;
   const int sub = r / BQ;
-  const uint32_t lane_off = (uint32_t)(wid * 32) << 16;
+  const uint32_t lane_off = (uint32_t)(q * 32) << 16;
   const uint32_t s_tmem = tmem + S::TMEM_S0 + s * BK + lane_off;
-  const uint32_t o_tmem = tmem + S::TMEM_O0 + s * D + lane_off;
-  const float tau = p.tau[hq];
-  const int mq = p.N / BQ, mkv = p.N / BK;
+  const uint32_t o_tmem = tmem + S::TMEM_O0 + s * D + c4 * QD + lane_off;
+  // [slot][quarter][row]: one buffer per slot. Consecutive blocks alternate
+  // slots, and the other slot's barrier in between orders this block's reads
+  // before the next write to the same buffer.
+  float* rowpart = &bars->xch[s * kRowSplit * 128];
 
-  float m = -INFINITY;   // running maximum, exp2 domain
-  float l = 0.f;         // running normaliser
-  bool failed = false;
-
-  for (int j = 0; j < nblk; ++j) {
-    const int buf = j & 1;
-    const bool ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[s], j & 1, abort_flag));
-    float sv[BK];
-    float rmax = -INFINITY;
-    if (ok) {
-      tc_fence_after();
-      uint32_t raw[BK];
-      if constexpr (BK == 128) tmem_ld_x128(s_tmem, raw);
-      else tmem_ld_x64(s_tmem, raw);
+  bool ok = true;
+  if (lane == 0) ok = mbar_wait(&bars->s_full[s], j & 1, abort_flag);
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  float sv[QC];
+  float pmax = -INFINITY;
+  if (ok) {
+    tc_fence_after();
+    uint32_t raw[QC];
+    if constexpr (QC == 64) tmem_ld_x64(s_tmem + c4 * QC, raw);
+    else if constexpr (QC == 32) tmem_ld_x32(s_tmem + c4 * QC, raw);
+    else tmem_ld_x16(s_tmem + c4 * QC, raw);
 #pragma unroll
-      for (int c = 0; c < BK; ++c) sv[c] = __uint_as_float(raw[c]);
-      if (CAUSAL && (j + 1) * BK - 1 > q0) {       // block straddles the causal boundary
+    for (int c = 0; c < QC; ++c) sv[c] = __uint_as_float(raw[c]);
+    const int k0 = j * BK + c4 * QC;
+    if (CAUSAL && k0 + QC - 1 > qrow) {          // this quarter reaches past the diagonal
 #pragma unroll
-        for (int c = 0; c < BK; ++c)
-          if (j * BK + c > qrow) sv[c] = -INFINITY;
-      }
-      float m0 = -INFINITY, m1 = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < BK; c += 4) {
-        m0 = max3(m0, sv[c], sv[c + 1]);
-        m1 = max3(m1, sv[c + 2], sv[c + 3]);
-      }
-      rmax = fmaxf(m0, m1);
+      for (int c = 0; c < QC; ++c)
+        if (k0 + c > qrow) sv[c] = -INFINITY;
     }
-    // Block maximum of each query tile: warp reduction, then across the tile's warps.
-    const float wmax = warp_max_redux(rmax);
-    if (lane == 0) bars->red[s][buf][wid] = wmax;
-    if (named_barrier_or(1 + s, 128, failed || !ok || *abort_flag)) {
-      failed = true;
-      break;
-    }
-    int code[S::NSUB];
-    bool keep_any = false;
+    float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll
-    for (int t = 0; t < S::NSUB; ++t) {
-      float bm = -INFINITY;
+    for (int c = 0; c < QC; c += 4) {
+      m0 = max3(m0, sv[c], sv[c + 1]);
+      m1 = max3(m1, sv[c + 2], sv[c + 3]);
+    }
+    pmax = fmaxf(m0, m1);
+  }
+  rowpart[c4 * 128 + r] = pmax;
+  // Gate: s_max * scale >= tau holds exactly when some thread's partial maximum
+  // does, so the barrier's OR over the query tile's threads is the decision.
+  // A thread that must stop raises this block's abort flag before arriving, so
+  // everyone reads the same value after the barrier.
+  if (failed || !ok || *abort_flag) ((volatile int*)bars->sm_abort)[j & 1] = 1;
+  const bool above = ok && (pmax * p.scale >= tau);
+  bool any_above[S::NSUB];
+  any_above[0] = named_barrier_or(1, 32 * kSoftmaxWarps, above && (S::NSUB == 1 || sub == 0));
+  if constexpr (S::NSUB == 2) any_above[1] = named_barrier_or(1, 32 * kSoftmaxWarps, above && sub == 1);
+  if (((volatile int*)bars->sm_abort)[j & 1]) return 2;
+  float rmax = -INFINITY;
 #pragma unroll
-      for (int u = t * (BQ / 32); u < (t + 1) * (BQ / 32); ++u) bm = fmaxf(bm, bars->red[s][buf][u]);
-      const int lo = q0 + t * BQ, hi = lo + BQ - 1;
-      const int k_lo = j * BK, k_hi = k_lo + BK - 1;
-      const bool visible = !CAUSAL || k_lo <= hi;
-      const bool diag = CAUSAL ? (visible && k_hi > lo) : (k_lo <= hi && k_hi >= lo);
-      code[t] = !visible ? 3 : diag ? 2 : ((bm * p.scale >= tau) ? 1 : 0);
-      keep_any |= (code[t] == 1 || code[t] == 2);
-    }
-    if (r == 0) {
-      if (WRITE_MASK) {
+  for (int u = 0; u < kRowSplit; ++u) rmax = fmaxf(rmax, rowpart[u * 128 + r]);
+  int code[S::NSUB];
+  bool keep_any = false;
 #pragma unroll
-        for (int t = 0; t < S::NSUB; ++t)
-          if (code[t] != 3)
-            p.mask[((size_t)(b * p.Hq + hq) * mq + (q0 / BQ + t)) * mkv + j] = (uint8_t)code[t];
-      }
-      // Publish the decision so the V tile (if kept) is fetched right away.
-      const int g = j % S::GR;
-      if (mbar_wait(&bars->gate_empty[s][g], ((j / S::GR) & 1) ^ 1, abort_flag)) {
-        ((volatile int*)&bars->gate_flag[s][g])[0] = keep_any ? 1 : 0;
-        mbar_arrive(&bars->gate_full[s][g]);
-      } else {
-        failed = true;
-      }
-      ((volatile int*)bars->p_keep)[s] = keep_any ? 1 : 0;
-    }
-    __syncwarp();
-    if (!keep_any) {                 // skipped by every tile of the slot: release S, nothing else
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->p_full[s]);
-      continue;
-    }
-
-    const int my_code = (S::NSUB == 1 || sub == 0) ? code[0] : code[S::NSUB - 1];
-    const bool my_keep = (my_code == 1 || my_code == 2);       // uniform within a warp
-    bool need_rescale = false;
-    float alpha = 1.f;
-    if (my_keep) {
-      const float mx = rmax * p.scale_log2;
-      if (mx > m + kRescaleThreshold) {      // also taken on the first finite maximum
-        if (m != -INFINITY) {
-          alpha = ex2_approx(m - mx);
-          need_rescale = true;
-        }
-        m = mx;
-      }
-      l *= alpha;
-    }
-    // P = 2^(s * log2(e)/sqrt(d) - m): half of the exponentials on the SFU (ex2),
-    // half as a polynomial on the FMA pipe, all other arithmetic in f32x2 pairs.
-    const bool live = my_keep && (m != -INFINITY);
-    const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
-    const float2 nm2 = make_float2(-m, -m);
-    float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
-    uint32_t pk[BK / 2];
+  for (int t = 0; t < S::NSUB; ++t) {
+    const int lo = q0 + t * BQ, hi = lo + BQ - 1;
+    const int k_lo = j * BK, k_hi = k_lo + BK - 1;
+    const bool visible = !CAUSAL || k_lo <= hi;
+    const bool diag = CAUSAL ? (visible && k_hi > lo) : (k_lo <= hi && k_hi >= lo);
+    code[t] = !visible ? 3 : diag ? 2 : (any_above[t] ? 1 : 0);
+    keep_any |= (code[t] == 1 || code[t] == 2);
+  }
+  if (warp == 0 && lane == 0) {
+    if (WRITE_MASK) {
+      const int mq = p.N / BQ, mkv = p.N / BK;
 #pragma unroll
-    for (int e = 0; e < BK / 2; e += 2) {
-      const float2 xa = __ffma2_rn(make_float2(sv[2 * e], sv[2 * e + 1]), sl2, nm2);
-      const float2 xb = __ffma2_rn(make_float2(sv[2 * e + 2], sv[2 * e + 3]), sl2, nm2);
-      const float2 pa = make_float2(ex2_approx(xa.x), ex2_approx(xa.y));
-      const float2 pb = exp2_poly2(xb);
-      acc0 = __fadd2_rn(acc0, pa);
-      acc1 = __fadd2_rn(acc1, pb);
-      pk[e] = pack_bf16x2(pa.x, pa.y);
-      pk[e + 1] = pack_bf16x2(pb.x, pb.y);
+      for (int t = 0; t < S::NSUB; ++t)
+        if (code[t] != 3)
+          p.mask[((size_t)(w.b * p.Hq + hq) * mq + (q0 / BQ + t)) * mkv + j] = (uint8_t)code[t];
     }
-    if (__any_sync(0xffffffffu, !live)) {   // rows this block does not update: P = 0
-      if (!live) {
-#pragma unroll
-        for (int e = 0; e < BK / 2; ++e) pk[e] = 0u;
-        acc0 = acc1 = make_float2(0.f, 0.f);
-      }
-    }
-    l += (acc0.x + acc0.y) + (acc1.x + acc1.y);
-    if constexpr (BK == 128) tmem_st_x64(s_tmem, pk);   // P (bf16 pairs) over the consumed S columns
-    else tmem_st_x32(s_tmem, pk);
-    tmem_st_wait();
-
-    // O_s is quiescent here: the commit that announced S_s(j) also covered PV_s(j-1).
-    if (__any_sync(0xffffffffu, need_rescale)) {
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
-        tmem_ld_x32(o_tmem + c * 32, o);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-        tmem_st_x32(o_tmem + c * 32, o);
-      }
-      tmem_st_wait();
-    }
+    // Publish the decision (no waiting) so the V tile, if kept, is fetched right away.
+    if (keep_any) atomicOr(&bars->gate_bits[s][j >> 5], 1u << (j & 31));
+    __threadfence_block();
+    ((volatile int*)bars->decided)[s] = j + 1;
+  }
+  if (!keep_any) {                 // skipped by every tile of the slot: release S, nothing else
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(&bars->p_full[s]);
+    return failed ? 1 : 0;
   }
 
-  // Epilogue: O / l -> bf16 rows, lse = ln-sum-exp over the kept set.
-  bool ok = !failed;
-  if (ok) ok = mbar_wait(&bars->o_done[s], 0, abort_flag);
-  ok = __all_sync(0xffffffffu, ok);
-  if (ok) {
-    tc_fence_after();
-    const float inv_l = 1.f / l;     // l > 0: every row keeps its diagonal block, which holds its own key
-    uint16_t* orow = p.out + ((size_t)(b * p.N + qrow) * p.Hq + hq) * D;
-#pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
-      uint32_t o[32];
-      tmem_ld_x32(o_tmem + c * 32, o);
-      uint32_t pk[16];
-#pragma unroll
-      for (int e = 0; e < 16; ++e)
-        pk[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
-      uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
-#pragma unroll
-      for (int v4 = 0; v4 < 4; ++v4) dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+  const int my_code = (S::NSUB == 1 || sub == 0) ? code[0] : code[S::NSUB - 1];
+  const bool my_keep = (my_code == 1 || my_code == 2);       // uniform within a warp
+  float m = s ? st.m[1] : st.m[0];
+  float l = s ? st.l[1] : st.l[0];
+  bool need_rescale = false;
+  float alpha = 1.f;
+  if (my_keep) {
+    const float mx = rmax * p.scale_log2;
+    if (mx > m + kRescaleThreshold) {      // also taken on the first finite maximum
+      if (m != -INFINITY) {
+        alpha = ex2_approx(m - mx);
+        need_rescale = true;
+      }
+      m = mx;
     }
-    if (p.lse != nullptr) p.lse[(size_t)(b * p.Hq + hq) * p.N + qrow] = (m + __log2f(l)) * 0.69314718055994531f;
+    l *= alpha;
+  }
+  // P = 2^(s * log2(e)/sqrt(d) - m): 5 of every 8 exponentials on the SFU (ex2),
+  // 3 as a polynomial on the FMA pipe, the rest of the arithmetic in f32x2 pairs.
+  // P (bf16 pairs) goes over S columns every thread of the slot has already read.
+  const bool live = my_keep && (m != -INFINITY);
+  const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
+  const float2 nm2 = make_float2(-m, -m);
+  float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+  uint32_t pk[QC / 2];
+#pragma unroll
+  for (int e = 0; e < QC / 2; ++e) {
+    const float2 x = __ffma2_rn(make_float2(sv[2 * e], sv[2 * e + 1]), sl2, nm2);
+    const bool poly = (e & 7) == 1 || (e & 7) == 4 || (e & 7) == 6;
+    const float2 pe = poly ? exp2_poly2(x) : make_float2(ex2_approx(x.x), ex2_approx(x.y));
+    pk[e] = pack_bf16x2(pe.x, pe.y);
+    if (e & 1) acc1 = __fadd2_rn(acc1, pe);
+    else acc0 = __fadd2_rn(acc0, pe);
+  }
+  if (__any_sync(0xffffffffu, !live) && !live) {   // rows this block does not update: P = 0
+#pragma unroll
+    for (int e = 0; e < QC / 2; ++e) pk[e] = 0u;
+  }
+  if (live) l += (acc0.x + acc0.y) + (acc1.x + acc1.y);
+  if constexpr (QC == 64) tmem_st_x32(s_tmem + c4 * (QC / 2), pk);
+  else if constexpr (QC == 32) tmem_st_x16(s_tmem + c4 * (QC / 2), pk);
+  else tmem_st_x8(s_tmem + c4 * (QC / 2), pk);
+  tmem_st_wait();
+
+  // O_s is quiescent here: the commit that announced S_s(j) also covered PV_s(j-1).
+  if (__any_sync(0xffffffffu, need_rescale)) {
+#pragma unroll
+    for (int c = 0; c < QD / 32 + (QD < 32); ++c) {
+      constexpr int W = QD < 32 ? QD : 32;
+      uint32_t o[W];
+      if constexpr (W == 32) tmem_ld_x32(o_tmem + c * 32, o);
+      else tmem_ld_x16(o_tmem, o);
+#pragma unroll
+      for (int e = 0; e < W; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+      if constexpr (W == 32) tmem_st_x32(o_tmem + c * 32, o);
+      else tmem_st_x16(o_tmem, o);
+    }
+    tmem_st_wait();
+  }
+  if (s) { st.m[1] = m; st.l[1] = l; } else { st.m[0] = m; st.l[0] = l; }
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(&bars->p_full[s]);
+  return failed ? 1 : 0;
+}
+
+// Epilogue of one slot: the four threads of each row combine their normalisers
+// through shared memory, then each writes its D/4 output columns; lse is the
+// natural-log logsumexp over the kept set.
+template <int D, int BQ, int BK, typename Bars>
+__device__ __forceinline__ void softmax_epilogue(const FwdParams& p, Bars* bars, uint32_t tmem, const FwdUnit& w,
+                                                 int s, SoftmaxRow<BK>& st, bool failed) {
+  using S = FwdShape<D, BQ, BK>;
+  constexpr int QD = D / kRowSplit;
+  volatile int* abort_flag = &bars->abort;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c4 = warp >> 2, q = warp & 3;
+  const int r = q * 32 + lane;
+  const int hq = s ? w.hq[1] : w.hq[0];
+  const int q0 = s ? w.q0[1] : w.q0[0];
+  const int qrow = q0 + r;
+  const float m = s ? st.m[1] : st.m[0];
+  const float l = s ? st.l[1] : st.l[0];
+  float* lpart = bars->xch;                  // [quarter][row], reused after the last block
+  // The exchange area may still be read for the last block's row maxima.
+  if (named_barrier_or(1, 32 * kSoftmaxWarps, failed || *abort_flag)) return;
+  lpart[c4 * 128 + r] = l;
+  const bool any_failed = named_barrier_or(1, 32 * kSoftmaxWarps, *abort_flag);
+  float l_row = 0.f;
+#pragma unroll
+  for (int u = 0; u < kRowSplit; ++u) l_row += lpart[u * 128 + r];
+  const bool again = named_barrier_or(1, 32 * kSoftmaxWarps, any_failed);   // everyone has read lpart
+  if (again) return;
+  bool ok = true;
+  if (lane == 0) ok = mbar_wait(&bars->o_done[s], 0, abort_flag);
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  if (!ok) return;
+  tc_fence_after();
+  const uint32_t o_tmem = tmem + S::TMEM_O0 + s * D + c4 * QD + ((uint32_t)(q * 32) << 16);
+  const float inv_l = 1.f / l_row;     // > 0: every row keeps its diagonal block, which holds its own key
+  uint16_t* orow = p.out + ((size_t)(w.b * p.N + qrow) * p.Hq + hq) * D + c4 * QD;
+#pragma unroll
+  for (int c = 0; c < QD / 32 + (QD < 32); ++c) {
+    constexpr int W = QD < 32 ? QD : 32;
+    uint32_t o[W];
+    if constexpr (W == 32) tmem_ld_x32(o_tmem + c * 32, o);
+    else tmem_ld_x16(o_tmem, o);
+    uint32_t pk[W / 2];
+#pragma unroll
+    for (int e = 0; e < W / 2; ++e)
+      pk[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
+    uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+    for (int v4 = 0; v4 < W / 8; ++v4) dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+  }
+  if (c4 == 0 && p.lse != nullptr)
+    p.lse[(size_t)(w.b * p.Hq + hq) * p.N + qrow] = (m + __log2f(l_row)) * 0.69314718055994531f;
+}
+
+template <int D, int BQ, int BK, bool CAUSAL, bool WRITE_MASK, typename Bars>
+__device__ __forceinline__ void softmax_role(const FwdParams& p, Bars* bars, uint32_t tmem, const FwdUnit& w) {
+  SoftmaxRow<BK> st;
+  bool failed = false, aborted = false;
+  const float tau0 = p.tau[w.hq[0]], tau1 = p.tau[w.hq[1]];
+  const int nblk = max(w.nblk[0], w.nblk[1]);
+  for (int j = 0; j < nblk && !aborted; ++j) {
+#pragma unroll 1
+    for (int s = 0; s < 2; ++s) {
+      if (j >= (s ? w.nblk[1] : w.nblk[0])) continue;
+      const int rv = softmax_block<D, BQ, BK, CAUSAL, WRITE_MASK>(p, bars, tmem, w, s, j, s ? tau1 : tau0, st, failed);
+      if (rv == 2) { aborted = true; break; }
+      failed = rv != 0;
+    }
+  }
+#pragma unroll 1
+  for (int s = 0; s < 2; ++s) {
+    if ((s ? w.nblk[1] : w.nblk[0]) == 0) continue;
+    softmax_epilogue<D, BQ, BK>(p, bars, tmem, w, s, st, failed || aborted);
   }
 }
 
@@ -493,10 +585,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     bsfa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
   using S = FwdShape<D, BQ, BK>;
-  using Bars = FwdBarriers<S::KS, S::VS, S::GR>;
+  using Bars = FwdBarriers<S::KS, S::VS>;
   static_assert(sizeof(Bars) <= S::BAR_BYTES, "barrier block");
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw;
   Bars* bars = reinterpret_cast<Bars*>(smem + S::OFF_BAR);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const FwdUnit w = decode_unit(p, blockIdx.x, CAUSAL, BK);
@@ -507,15 +599,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < S::VS; ++i) { mbar_init(&bars->v_full[i], 1); mbar_init(&bars->v_empty[i], 1); }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars->s_full[i], 1);
-      mbar_init(&bars->p_full[i], 4);          // one arrival per softmax warp
+      mbar_init(&bars->p_full[i], kSoftmaxWarps);   // one arrival per softmax warp
       mbar_init(&bars->o_done[i], 1);
-      for (int g = 0; g < S::GR; ++g) { mbar_init(&bars->gate_full[i][g], 1); mbar_init(&bars->gate_empty[i][g], 1); }
+      bars->sm_abort[i] = 0;
+      bars->decided[i] = 0;
     }
+    for (int i = 0; i < 2 * (kMaxKeyBlocks / 32); ++i) (&bars->gate_bits[0][0])[i] = 0u;
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
     fence_mbar_init();
   }
-  if (warp == 8) {
+  // The 128-byte swizzle and the descriptors assume a 1024-byte aligned base.
+  if ((smem_u32(smem) & 1023u) != 0) {
+    if (threadIdx.x == 0) atomicOr(p.status, 2);
+    return;
+  }
+  if (warp == kSoftmaxWarps) {
     tmem_alloc(&bars->tmem_base, S::TMEM_COLS);
     tmem_relinquish();
     tc_fence_before();
@@ -524,22 +623,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 
-  if (warp < 8) {
+  if (warp < kSoftmaxWarps) {
     regs_increase<kSoftmaxRegs>();
     softmax_role<D, BQ, BK, CAUSAL, WRITE_MASK>(p, bars, tmem, w);
   } else {
     regs_decrease<kProducerRegs>();
     if (lane == 0) {
-      if (warp == 8) kq_producer<D, BQ, BK>(&tm_q, &tm_k, smem, bars, w);
-      else if (warp == 9) mma_issuer<D, BQ, BK>(smem, bars, tmem, w);
-      else if (warp == 10) v_producer<D, BQ, BK>(&tm_v, smem, bars, w);
+      if (warp == kSoftmaxWarps) kq_producer<D, BQ, BK>(&tm_q, &tm_k, smem, bars, w);
+      else if (warp == kSoftmaxWarps + 1) mma_issuer<D, BQ, BK>(smem, bars, tmem, w);
+      else if (warp == kSoftmaxWarps + 2) v_producer<D, BQ, BK>(&tm_v, smem, bars, w);
     }
     __syncwarp();
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == kSoftmaxWarps) {
     tc_fence_after();
     tmem_dealloc(tmem, S::TMEM_COLS);
   }
