@@ -181,7 +181,9 @@ __device__ __forceinline__ void kq_producer(const CUtensorMap* tm_q, const CUten
     drain_wait(&bars->k_full[t % S::KS], (t / S::KS) & 1);
 }
 
-// Bounded spin until slot s's gate decision for block j is published.
+// Bounded wait until slot s's gate decision for block j is published. The
+// thread sleeps between looks: a tight shared-memory spin would steal the
+// bandwidth the QK^T MMAs (both operands in shared memory) depend on.
 template <typename Bars>
 __device__ __forceinline__ bool wait_decided(Bars* bars, int s, int j) {
   volatile int* decided = &bars->decided[s];
@@ -189,9 +191,8 @@ __device__ __forceinline__ bool wait_decided(Bars* bars, int s, int j) {
   if (*decided > j) return true;
   const uint64_t t0 = global_timer_ns();
   for (;;) {
-#pragma unroll 1
-    for (int i = 0; i < 256; ++i)
-      if (*decided > j) return true;
+    __nanosleep(64);
+    if (*decided > j) return true;
     if (*abort_flag) return false;
     if (global_timer_ns() - t0 > kWaitTimeoutNs) {
       *abort_flag = 1;
@@ -454,8 +455,8 @@ __device__ __forceinline__ int softmax_block(const FwdParams& p, Bars* bars, uin
     }
     l *= alpha;
   }
-  // P = 2^(s * log2(e)/sqrt(d) - m): 5 of every 8 exponentials on the SFU (ex2),
-  // 3 as a polynomial on the FMA pipe, the rest of the arithmetic in f32x2 pairs.
+  // P = 2^(s * log2(e)/sqrt(d) - m): 3 of every 4 exponentials on the SFU (ex2),
+  // 1 as a polynomial on the FMA pipe, the rest of the arithmetic in f32x2 pairs.
   // P (bf16 pairs) goes over S columns every thread of the slot has already read.
   const bool live = my_keep && (m != -INFINITY);
   const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
@@ -465,7 +466,7 @@ __device__ __forceinline__ int softmax_block(const FwdParams& p, Bars* bars, uin
 #pragma unroll
   for (int e = 0; e < QC / 2; ++e) {
     const float2 x = __ffma2_rn(make_float2(sv[2 * e], sv[2 * e + 1]), sl2, nm2);
-    const bool poly = (e & 7) == 1 || (e & 7) == 4 || (e & 7) == 6;
+    const bool poly = (e & 3) == 3;
     const float2 pe = poly ? exp2_poly2(x) : make_float2(ex2_approx(x.x), ex2_approx(x.y));
     pk[e] = pack_bf16x2(pe.x, pe.y);
     if (e & 1) acc1 = __fadd2_rn(acc1, pe);
