@@ -86,6 +86,16 @@ bsfa_status bsfa_validate(int B, int Hq, int Hkv, int N, int D, int Bq, int Bk, 
  */
 bsfa_status bsfa_get_status(void* stream);
 
+/*
+ * bsfa_selftest_lost_arrival - exercise the failure path on the device: one
+ * thread waits, through the forward kernel's bounded wait, on a barrier that
+ * nothing arrives on (the shape of a lost arrival). After the wait's time limit
+ * (about 2 s) the kernel sets the device status word and exits normally; no
+ * trap, the context stays usable. Asynchronous on `stream`; the next
+ * bsfa_get_status(stream) returns BSFA_ERR_DEVICE_TIMEOUT.
+ */
+bsfa_status bsfa_selftest_lost_arrival(void* stream);
+
 /* bsfa_status_string - a static, human-readable name for a status code. */
 const char* bsfa_status_string(bsfa_status s);
 

@@ -25,7 +25,8 @@ BSFA_ERR_UNSUPPORTED = 2
 BSFA_ERR_CUDA = 3
 BSFA_ERR_DEVICE_TIMEOUT = 4
 
-EXPORTED = ("bsfa_forward", "bsfa_validate", "bsfa_get_status", "bsfa_status_string", "bsfa_last_error")
+EXPORTED = ("bsfa_forward", "bsfa_validate", "bsfa_get_status", "bsfa_selftest_lost_arrival", "bsfa_status_string",
+            "bsfa_last_error")
 
 _lib = None
 
@@ -51,6 +52,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.bsfa_validate.restype = i
     lib.bsfa_get_status.argtypes = [vp]
     lib.bsfa_get_status.restype = i
+    lib.bsfa_selftest_lost_arrival.argtypes = [vp]
+    lib.bsfa_selftest_lost_arrival.restype = i
     lib.bsfa_status_string.argtypes = [i]
     lib.bsfa_status_string.restype = ctypes.c_char_p
     lib.bsfa_last_error.argtypes = []
@@ -88,6 +91,10 @@ def bsfa_validate(B, Hq, Hkv, N, D, Bq, Bk, causal) -> int:
 
 def bsfa_get_status(stream=None) -> int:
     return load().bsfa_get_status(_stream(stream))
+
+
+def bsfa_selftest_lost_arrival(stream=None) -> int:
+    return load().bsfa_selftest_lost_arrival(_stream(stream))
 
 
 def bsfa_status_string(status: int) -> str:

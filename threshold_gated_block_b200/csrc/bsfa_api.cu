@@ -87,6 +87,20 @@ bool encode_bnhd(CUtensorMap* map, const void* ptr, int B, int N, int H, int D, 
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// One thread waits, through the same bounded wait the forward kernel uses, on an
+// mbarrier that nothing will ever arrive on. The wait gives up after its time
+// limit and the kernel reports through the status word, exactly as a forward
+// kernel that lost an arrival would.
+__global__ void selftest_lost_arrival_kernel(int* status) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x != 0) return;
+  bsfa::mbar_init(&bar, 1);
+  bsfa::fence_mbar_init();
+  abort_flag = 0;
+  if (!bsfa::mbar_wait(&bar, 0, &abort_flag)) atomicOr(status, 1);
+}
+
 }  // namespace
 
 extern "C" {
@@ -180,6 +194,19 @@ bsfa_status bsfa_get_status(void* stream) {
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(clear status word)");
     return fail(BSFA_ERR_DEVICE_TIMEOUT, "a kernel gave up on a bounded wait (status word 0x%x)", word);
   }
+  return BSFA_OK;
+}
+
+bsfa_status bsfa_selftest_lost_arrival(void* stream) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  int* status_ptr = nullptr;
+  bsfa_status st = device_setup(dev, &status_ptr);
+  if (st != BSFA_OK) return st;
+  selftest_lost_arrival_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(status_ptr);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "self-test launch");
   return BSFA_OK;
 }
 
