@@ -20,8 +20,18 @@ def _is_valid(r: int, c: int, causal: bool) -> bool:
     return c <= r if causal else True
 
 
+def _threshold(tau, hq: int, i: int) -> float:
+    """tau[hq] when it is a number; else the per-tile list tau[hq], whose last
+    entry serves every tile past its end (§4.1, App. B.3 "Threshold tensor")."""
+    t = tau[hq]
+    if isinstance(t, (list, tuple)):
+        return t[i] if i < len(t) else t[len(t) - 1]
+    return t
+
+
 def brute_forward(q, k, v, tau, Bq: int, Bk: int, causal: bool):
-    """q: float [B][N][Hq][D]; k, v: float [B][N][Hkv][D]; tau: [Hq].
+    """q: float [B][N][Hq][D]; k, v: float [B][N][Hkv][D]; tau: [Hq] numbers, or
+    [Hq] lists of per-query-tile thresholds.
 
     Returns (out [B][N][Hq][D], lse [B][Hq][N], codes {(b, hq, i, j): code}).
     """
@@ -49,7 +59,6 @@ def brute_forward(q, k, v, tau, Bq: int, Bk: int, causal: bool):
                 for j in range(mkv):
                     cols = range(j * Bk, min((j + 1) * Bk, N))
                     any_valid = False
-                    any_invalid = False
                     best = -math.inf
                     for r in rows:
                         for c in cols:
@@ -57,18 +66,20 @@ def brute_forward(q, k, v, tau, Bq: int, Bk: int, causal: bool):
                                 any_valid = True
                                 if s[r][c] > best:
                                     best = s[r][c]
-                            else:
-                                any_invalid = True
                     if not any_valid:
                         codes[(b, hq, i, j)] = 3
                         continue
+                    # Forced blocks are found on the full-size tile and block, as if
+                    # the sequence were padded to whole tiles.
+                    full_rows = range(i * Bq, (i + 1) * Bq)
+                    full_cols = range(j * Bk, (j + 1) * Bk)
                     if causal:
-                        forced = any_invalid
+                        forced = any(not _is_valid(r, c, True) for r in full_rows for c in full_cols)
                     else:
-                        forced = any(c in rows for c in cols)
+                        forced = any(c in full_rows for c in full_cols)
                     if forced:
                         codes[(b, hq, i, j)] = 2
-                    elif best >= tau[hq]:
+                    elif best >= _threshold(tau, hq, i):
                         codes[(b, hq, i, j)] = 1
                     else:
                         codes[(b, hq, i, j)] = 0

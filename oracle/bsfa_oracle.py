@@ -34,10 +34,12 @@ design notes):
   * s_max is one scalar per (query tile, key block), the maximum over every
     valid entry of the block;
   * causal: a block is visible when some entry is valid (key <= query); it is
-    "diagonal" when it is visible and also holds an invalid entry;
+    "diagonal" when it is visible and also holds an invalid entry, the tile and
+    block taken at full size (as if padded, App. B.3);
     non-causal: a block is "diagonal" when its key range overlaps the tile's
     query range;
-  * tau is one float per query head;
+  * tau is one float per query head, or a per-position table [Hq, M] (one
+    value per query tile; tiles past the table's end reuse its last column);
   * GQA: query head h reads KV head h // (Hq / Hkv);
   * lse is the natural-log logsumexp, laid out [B, Hq, N];
   * keys at index >= N are invalid (an unaligned tail is never read).
@@ -73,6 +75,21 @@ def gate_keep(smax: float, tau: float) -> bool:
     return smax >= tau
 
 
+def tile_tau(tau, hq: int, i: int) -> float:
+    """Threshold of query tile i of head hq.
+
+    §4.1 gates block (i, j) against a threshold indexed by layer, head and query
+    position; App. B.3 "Threshold tensor" stores ceil(N_max / B_M) positions per
+    head, and a sequence longer than N_max reuses the threshold of the last
+    calibrated position. ``tau`` is one layer's slice: either [Hq] (one value per
+    head) or [Hq, M] (one value per head and query tile).
+    """
+    t = np.asarray(tau, dtype=np.float64)
+    if t.ndim == 1:
+        return float(t[hq])
+    return float(t[hq, min(i, t.shape[1] - 1)])
+
+
 def kv_head(hq: int, Hq: int, Hkv: int) -> int:
     """GQA: contiguous groups of Hq/Hkv query heads share one KV head."""
     return hq // (Hq // Hkv)
@@ -96,14 +113,21 @@ def block_visible(i: int, j: int, Bq: int, Bk: int, N: int, causal: bool) -> boo
 
 
 def block_diagonal(i: int, j: int, Bq: int, Bk: int, N: int, causal: bool) -> bool:
-    """The blocks that bypass the gate (§4.1, "Diagonal blocks bypass the gate")."""
+    """The blocks that bypass the gate (§4.1, "Diagonal blocks bypass the gate").
+
+    Judged on the full tile and block, [i*Bq, (i+1)*Bq) x [j*Bk, (j+1)*Bk), as if an
+    unaligned sequence were padded to whole tiles (App. B.3 "Practical
+    considerations"): a visible block is diagonal when it holds, or would hold, a
+    key later than the tile's first query (causal), or when its key range overlaps
+    the tile's query range (bidirectional). The block holding a row's own key is
+    therefore always forced, also for a last tile cut down to a single row.
+    """
     if not block_visible(i, j, Bq, Bk, N, causal):
         return False
-    r0, r1 = tile_rows(i, Bq, N)
-    c0, c1 = block_cols(j, Bk, N)
+    r0, c0 = i * Bq, j * Bk
     if causal:
-        return c1 - 1 > r0          # holds at least one key later than some query
-    return c0 < r1 and c1 > r0       # key range overlaps the query range
+        return c0 + Bk - 1 > r0
+    return c0 < r0 + Bq and c0 + Bk > r0
 
 
 def valid_mask(r0: int, r1: int, ncols: int, causal: bool) -> np.ndarray:
@@ -170,7 +194,8 @@ def forward_tile(q_bits, k_bits, v_bits, tau, b: int, hq: int, i: int, Bq: int, 
                  causal: bool, flip=(), with_output: bool = True) -> dict:
     """The BSFA result for one query tile (b, hq, i).
 
-    q_bits: uint16 [B, N, Hq, D]; k_bits, v_bits: uint16 [B, N, Hkv, D]; tau: per-head floats.
+    q_bits: uint16 [B, N, Hq, D]; k_bits, v_bits: uint16 [B, N, Hkv, D]; tau: [Hq] or [Hq, M]
+    (see ``tile_tau``).
     Returns out [rows, D], lse [rows], codes [M_KV], smax [M_KV] (NaN where not visible).
     """
     B, N, Hq, D = q_bits.shape
@@ -182,7 +207,7 @@ def forward_tile(q_bits, k_bits, v_bits, tau, b: int, hq: int, i: int, Bq: int, 
     kmat = widen_bf16(k_bits[b, :ncols, g, :])
     S = tile_scores(qi, kmat, D)
     valid = valid_mask(r0, r1, ncols, causal)
-    codes, smax = tile_block_codes(S, valid, i, float(tau[hq]), Bq, Bk, N, causal, flip)
+    codes, smax = tile_block_codes(S, valid, i, tile_tau(tau, hq, i), Bq, Bk, N, causal, flip)
     res = {"codes": codes, "smax": smax, "rows": (r0, r1)}
     if with_output:
         vmat = widen_bf16(v_bits[b, :ncols, g, :])

@@ -2,10 +2,12 @@
 
 Every mutation below swaps one helper of ``oracle.bsfa_oracle`` for a wrong
 version (a dropped or wrong score scale, a strict comparison at the gate, an
-inverted gate, no diagonal bypass, a wrong GQA head map, a normaliser that
-counts skipped blocks, a gate on unscaled scores or on the block minimum). The pin
-battery (hand-derived closed forms, the scalar brute force, and the tau = -inf /
-tau = +inf library cases) must fail for each of them.
+inverted gate, no diagonal bypass, a diagonal judged on the cut-down last tile,
+a wrong GQA head map, a normaliser that counts skipped blocks, a gate on unscaled
+scores or on the block minimum, a per-position threshold table read at the wrong
+column). The pin battery (hand-derived closed forms, the scalar brute force on
+aligned and ragged sequences with per-head and per-tile thresholds, and the
+tau = -inf library case) must fail for each of them.
 """
 import json
 import math
@@ -54,6 +56,16 @@ def _battery(golden_dir) -> bool:
             ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=causal)
             if not np.allclose(r["out"], ref.permute(0, 2, 1, 3).numpy(), atol=1e-12, rtol=0):
                 return False
+        # ragged end (last tile of one row) with a per-tile table shorter than M_Q
+        x = make_inputs(custom_config(N=65, D=8, Hq=2, Hkv=1, Bq=16, Bk=16, causal=True, seed=98))
+        table = [[2.9, 2.2, 2.6], [2.4, 3.0, 2.5]]
+        r = O.forward(x["q"], x["k"], x["v"], table, 16, 16, True)
+        qf, kf, vf = (O.widen_bf16(x[n]).tolist() for n in "qkv")
+        out, lse, codes = brute.brute_forward(qf, kf, vf, table, 16, 16, True)
+        if any(r["codes"][key] != c for key, c in codes.items()):
+            return False
+        if not (np.allclose(r["out"], out, atol=1e-12, rtol=0) and np.allclose(r["lse"], lse, atol=1e-12, rtol=0)):
+            return False
     return True
 
 
@@ -71,6 +83,24 @@ def _inverted_gate(smax, tau):
 
 def _no_diagonal(i, j, Bq, Bk, N, causal):
     return False
+
+
+def _diagonal_on_clipped_tile(i, j, Bq, Bk, N, causal):
+    if not O.block_visible(i, j, Bq, Bk, N, causal):
+        return False
+    r0, r1 = O.tile_rows(i, Bq, N)
+    c0, c1 = O.block_cols(j, Bk, N)
+    return (c1 - 1 > r0) if causal else (c0 < r1 and c1 > r0)
+
+
+def _table_wraps(tau, hq, i):
+    t = np.asarray(tau, dtype=np.float64)
+    return float(t[hq]) if t.ndim == 1 else float(t[hq, i % t.shape[1]])
+
+
+def _table_first_column(tau, hq, i):
+    t = np.asarray(tau, dtype=np.float64)
+    return float(t[hq]) if t.ndim == 1 else float(t[hq, 0])
 
 
 def _wrong_gqa(hq, Hq, Hkv):
@@ -107,6 +137,9 @@ MUTATIONS = {
     "strict comparison at the gate": ("gate_keep", _strict_gate),
     "inverted gate": ("gate_keep", _inverted_gate),
     "no diagonal bypass": ("block_diagonal", _no_diagonal),
+    "diagonal judged on the cut-down last tile": ("block_diagonal", _diagonal_on_clipped_tile),
+    "threshold table wraps instead of reusing its last column": ("tile_tau", _table_wraps),
+    "threshold table read at its first column only": ("tile_tau", _table_first_column),
     "wrong GQA head map": ("kv_head", _wrong_gqa),
     "normaliser counts skipped blocks": ("tile_softmax", _normaliser_counts_skipped),
     "gate compares the unscaled score": ("tile_block_codes", _gate_on_unscaled_scores),

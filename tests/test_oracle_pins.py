@@ -79,6 +79,11 @@ BRUTE_CASES = [
     (48, 8, 2, 2, 16, 16, False),
     (64, 8, 4, 2, 32, 16, False),
     (128, 8, 2, 1, 32, 32, True),
+    # ragged sequence ends: a last tile of one row, partial key blocks
+    (65, 8, 2, 1, 16, 16, True),
+    (81, 8, 4, 2, 32, 16, True),
+    (50, 8, 2, 1, 16, 32, False),
+    (97, 16, 2, 2, 32, 32, False),
 ]
 
 
@@ -100,6 +105,42 @@ def test_oracle_matches_scalar_brute_force(N, D, Hq, Hkv, Bq, Bk, causal):
     assert (r["codes"] == O.CODE_SKIPPED).any() and (r["codes"] == O.CODE_KEPT).any()
     np.testing.assert_allclose(r["out"], np.array(out), rtol=0, atol=1e-12)
     np.testing.assert_allclose(r["lse"], np.array(lse), rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("N,causal", [(96, True), (81, True), (70, False)])
+def test_per_tile_thresholds_match_brute_force(N, causal):
+    """A [Hq, T] table: tile i of head h uses column min(i, T-1) (§4.1, App. B.3)."""
+    Bq = Bk = 16
+    cfg = custom_config(N=N, D=8, Hq=2, Hkv=1, Bq=Bq, Bk=Bk, causal=causal, seed=N)
+    x = make_inputs(cfg)
+    mq = -(-N // Bq)
+    rng = np.random.default_rng(N)
+    table = rng.uniform(2.0, 3.2, size=(2, mq - 2))          # shorter than M_Q: the last column is reused
+    r = O.forward(x["q"], x["k"], x["v"], table, Bq, Bk, causal)
+    qf, kf, vf = (O.widen_bf16(x[n]).tolist() for n in "qkv")
+    out, lse, codes = brute.brute_forward(qf, kf, vf, [list(row) for row in table], Bq, Bk, causal)
+    for key, c in codes.items():
+        assert r["codes"][key] == c, key
+    assert (r["codes"] == O.CODE_SKIPPED).any() and (r["codes"] == O.CODE_KEPT).any()
+    np.testing.assert_allclose(r["out"], np.array(out), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(r["lse"], np.array(lse), rtol=0, atol=1e-12)
+    # a per-head vector and a one-column table are the same thresholds
+    per_head = O.forward(x["q"], x["k"], x["v"], table[:, 0], Bq, Bk, causal)
+    one_col = O.forward(x["q"], x["k"], x["v"], table[:, :1], Bq, Bk, causal)
+    assert np.array_equal(per_head["codes"], one_col["codes"])
+
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("N", [33, 65, 97])
+def test_every_row_keeps_its_own_key_at_ragged_ends(N, causal):
+    """At tau=+inf only forced blocks remain; with N = 1 (mod Bq) the last tile has
+    one row, and the block holding that row's key must still be forced."""
+    cfg = custom_config(N=N, D=8, Hq=1, Hkv=1, Bq=32, Bk=32, causal=causal, seed=N)
+    x = make_inputs(cfg)
+    r = O.forward(x["q"], x["k"], x["v"], [np.inf], 32, 32, causal)
+    assert np.isfinite(r["lse"]).all() and np.isfinite(r["out"]).all()
+    for row in range(N):
+        assert r["codes"][0, 0, row // 32, row // 32] == O.CODE_FORCED
 
 
 # ----------------------------------------------------------------------------- library special cases
