@@ -40,6 +40,9 @@ from threshold_gated_block_b200.inputs import CONFIGS, make_inputs, sample_tiles
 METRIC = "prefill-attention TFLOP/s (dense-equivalent)"
 UNIT = "TFLOP/s"
 TAUS = os.path.join(ROOT, "tests", "golden", "taus.json")
+TAU_TABLES = os.path.join(ROOT, "tests", "golden", "tau_tables.json")
+# Workloads that share one layer type share its per-position threshold table.
+TABLE_FOR = {"c2": "c2", "c3": "c2", "c4": "c2"}
 PEAKS = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC = os.path.join(ROOT, "profiles", "bsfa_fwd_c2_traffic.txt")
 KERNEL_SOURCES = ["ptx.cuh", "bsfa_fwd_kernel.cuh", "bsfa_launch.cuh", "bsfa_fwd_d64.cu", "bsfa_fwd_d128.cu",
@@ -55,23 +58,33 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="c2")
     ap.add_argument("--skip", type=float, default=None, help="target skip fraction (a stored calibration)")
+    ap.add_argument("--tau-table", type=int, default=None, metavar="K",
+                    help="gate with the stored per-position (fixed-k) table level that keeps K blocks per tile")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU-oracle baseline")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
 
 
 def workload(args):
+    """(config, threshold description, thresholds): per head [Hq] or per position [Hq, T]."""
     cfg = CONFIGS[args.config]
+    if args.tau_table is not None:
+        with open(TAU_TABLES) as f:
+            spec = json.load(f)[TABLE_FOR[cfg.name]]
+        level = spec["ks"].index(args.tau_table)
+        desc = {"tau": "per-position table", "k": args.tau_table, "table_n_max": spec["n_max"],
+                "calib_seeds": spec["calib_seeds"]}
+        return cfg, desc, spec["table"][level]
     p = cfg.skips[0] if args.skip is None else args.skip
     with open(TAUS) as f:
         taus = json.load(f)[cfg.name]["taus"][str(float(p))]
-    return cfg, p, taus
+    return cfg, {"tau": "per head", "target_skip": p}, taus
 
 
-def config_record(cfg, p, achieved=None):
+def config_record(cfg, tau_desc, achieved=None):
     rec = {"workload": f"{cfg.name}: {cfg.description}", "B": cfg.B, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "D": cfg.D,
            "N": cfg.N, "Bq": cfg.Bq, "Bk": cfg.Bk, "causal": cfg.causal, "inputs": cfg.kind,
-           "target_skip": p, "l2": "flushed between steps (256 MB memset outside the timed events)"}
+           **tau_desc, "l2": "flushed between steps (256 MB memset outside the timed events)"}
     if achieved is not None:
         rec["achieved_skip"] = achieved
     return rec
@@ -269,8 +282,12 @@ def run_ours(args):
     stream = torch.cuda.current_stream(dev)
 
     def step(t):
-        st = bsfa.bsfa_forward(q, k, v, t, out, lse, None, cfg.B, cfg.Hq, cfg.Hkv, cfg.N, cfg.D, cfg.Bq, cfg.Bk,
-                               cfg.causal, stream)
+        if t.dim() == 1:
+            st = bsfa.bsfa_forward(q, k, v, t, out, lse, None, cfg.B, cfg.Hq, cfg.Hkv, cfg.N, cfg.D, cfg.Bq, cfg.Bk,
+                                   cfg.causal, stream)
+        else:
+            st = bsfa.bsfa_forward_tau_table(q, k, v, t, t.shape[1], out, lse, None, cfg.B, cfg.Hq, cfg.Hkv, cfg.N,
+                                             cfg.D, cfg.Bq, cfg.Bk, cfg.causal, stream)
         if st != bsfa.BSFA_OK:
             raise RuntimeError(bsfa.bsfa_last_error())
 

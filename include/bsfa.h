@@ -11,7 +11,9 @@
  * query tile's kept key set.
  *
  * Definitions used by every entry point:
- *   - Query tile i holds rows [i*Bq, (i+1)*Bq); key block j holds keys [j*Bk, (j+1)*Bk).
+ *   - Query tile i holds rows [i*Bq, min((i+1)*Bq, N)); key block j holds keys
+ *     [j*Bk, min((j+1)*Bk, N)). There are M_Q = ceil(N/Bq) tiles and
+ *     M_KV = ceil(N/Bk) blocks (App. B.2); N need not be a multiple of either.
  *   - Causal: key c is valid for query r when c <= r. A block is visible when some
  *     entry is valid; it is diagonal (gate bypassed) when it is visible and also
  *     holds an invalid entry. Non-causal ("bidirectional", App. B.3): the diagonal
@@ -53,7 +55,7 @@ typedef enum {
  *   out        bf16 [B, N, Hq, D], contiguous, device memory, 16-byte aligned (written)
  *   lse        fp32 [B, Hq, N], device memory, natural-log logsumexp over each row's kept
  *              set (written); NULL skips it
- *   block_mask uint8 [B, Hq, N/Bq, N/Bk], device memory (written); NULL turns the debug
+ *   block_mask uint8 [B, Hq, M_Q, M_KV], device memory (written); NULL turns the debug
  *              output off. Codes: 0 skipped by the gate, 1 kept by the gate, 2 diagonal
  *              (forced keep), 3 not visible. The library fills it with 3 first.
  *   B, Hq, Hkv, N, D   sizes; Hq % Hkv == 0
@@ -61,8 +63,10 @@ typedef enum {
  *   causal     nonzero for causal prefill, zero for bidirectional attention
  *   stream     a cudaStream_t (NULL = the legacy default stream)
  *
- * Supported: D in {64, 128}; Bq, Bk in {64, 128}; N a positive multiple of 128
- * with at most 4096 key blocks (N / Bk <= 4096); an sm_100 device. The caller owns every buffer; results are valid once the
+ * Supported: D in {64, 128}; Bq, Bk in {64, 128}; any N >= 1 with at most 4096
+ * key blocks (M_KV <= 4096); an sm_100 device. Rows and keys past N inside the
+ * last tile or block are padding: they never enter a block maximum or a softmax,
+ * and no output row past N is written. The caller owns every buffer; results are valid once the
  * stream has reached the call. Returns BSFA_OK once the kernel is enqueued;
  * argument errors are returned before any CUDA call is made. A kernel that gives
  * up on a bounded internal wait leaves `out` undefined and sets the device
@@ -71,6 +75,27 @@ typedef enum {
 bsfa_status bsfa_forward(const void* q, const void* k, const void* v, const float* tau, void* out, float* lse,
                          uint8_t* block_mask, int B, int Hq, int Hkv, int N, int D, int Bq, int Bk, int causal,
                          void* stream);
+
+/*
+ * bsfa_forward_tau_table - bsfa_forward with one threshold per (query head,
+ * query tile): the per-position thresholds of §4.1 / §4.2 ("thresholds
+ * calibrated per (layer, head, position)").
+ *
+ *   tau_table  fp32 [Hq, tau_tiles], device memory, row-major (read). Query tile i
+ *              of head h is gated against tau_table[h * tau_tiles + min(i, tau_tiles - 1)]:
+ *              a sequence longer than the calibrated length reuses the last
+ *              calibrated position (App. B.3 "Practical considerations"). One layer
+ *              and sparsity level of the paper's table T[S, L, H, ceil(N_max/B_M)] is
+ *              the contiguous slice T[level, layer], with tau_tiles = ceil(N_max/B_M);
+ *              the table must be calibrated with the same Bq.
+ *   tau_tiles  number of calibrated query tiles per head, >= 1
+ *
+ * Every other argument, the supported set and the error behaviour are those of
+ * bsfa_forward; tau_tiles <= 0 returns BSFA_ERR_INVALID_ARG.
+ */
+bsfa_status bsfa_forward_tau_table(const void* q, const void* k, const void* v, const float* tau_table, int tau_tiles,
+                                   void* out, float* lse, uint8_t* block_mask, int B, int Hq, int Hkv, int N, int D,
+                                   int Bq, int Bk, int causal, void* stream);
 
 /*
  * bsfa_validate - the shape checks of bsfa_forward, host only (no CUDA call).

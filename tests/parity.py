@@ -79,12 +79,13 @@ def compare_tiles(x: dict, tau, Bq: int, Bk: int, causal: bool, gpu: dict, tiles
     rep = report or Report()
     tau = np.asarray(tau, dtype=np.float64)
     for (b, hq, i) in tiles:
+        tau_i = O.tile_tau(tau, hq, i)
         t = O.forward_tile(x["q"], x["k"], x["v"], tau, b, hq, i, Bq, Bk, causal)
         flip = ()
         if gpu["mask"] is not None:
             gm = gpu["mask"][b, hq, i]
             gated = np.isin(t["codes"], (O.CODE_SKIPPED, O.CODE_KEPT))
-            near = gated & (np.abs(t["smax"] - tau[hq]) <= NEAR_TAU)
+            near = gated & (np.abs(t["smax"] - tau_i) <= NEAR_TAU)
             rep.near_tau += int(near.sum())
             differ = gm != t["codes"]
             flip = tuple(int(j) for j in np.nonzero(differ & near)[0])
@@ -104,4 +105,4 @@ def compare_tiles(x: dict, tau, Bq: int, Bk: int, causal: bool, gpu: dict, tiles
 
 
 def all_tiles(B, Hq, N, Bq):
-    return [(b, h, i) for b in range(B) for h in range(Hq) for i in range(N // Bq)]
+    return [(b, h, i) for b in range(B) for h in range(Hq) for i in range(-(-N // Bq))]

@@ -51,7 +51,9 @@ def test_status_strings(lib):
     ((1, 32, 8, 8192, 96, 128, 128, 1), bsfa.BSFA_ERR_UNSUPPORTED),
     ((1, 32, 8, 8192, 128, 32, 128, 1), bsfa.BSFA_ERR_UNSUPPORTED),
     ((1, 32, 8, 8192, 128, 128, 256, 1), bsfa.BSFA_ERR_UNSUPPORTED),
-    ((1, 32, 8, 8000, 128, 128, 128, 1), bsfa.BSFA_ERR_UNSUPPORTED),
+    ((1, 32, 8, 8000, 128, 128, 128, 1), bsfa.BSFA_OK),          # ragged end
+    ((1, 2, 2, 1, 64, 64, 128, 0), bsfa.BSFA_OK),               # a single token
+    ((1, 8, 8, 4096 * 64 + 1, 64, 64, 64, 1), bsfa.BSFA_ERR_UNSUPPORTED),   # ceil(N/Bk) = 4097
     ((1024, 64, 8, 65536, 128, 128, 128, 1), bsfa.BSFA_ERR_UNSUPPORTED),
     ((1, 8, 8, 4096 * 64, 64, 64, 64, 1), bsfa.BSFA_OK),
     ((1, 8, 8, 4096 * 64 + 128, 64, 64, 64, 1), bsfa.BSFA_ERR_UNSUPPORTED),
@@ -71,5 +73,15 @@ def test_forward_rejects_bad_pointers_without_touching_cuda(lib):
     # misaligned lse
     assert bsfa.bsfa_forward(16, 16, 16, 16, 16, 2, None, *shape, None) == bsfa.BSFA_ERR_INVALID_ARG
     # unsupported shape wins before pointer checks
-    assert bsfa.bsfa_forward(None, None, None, None, None, None, None, 1, 2, 2, 500, 64, 64, 64, 1, None) \
+    assert bsfa.bsfa_forward(None, None, None, None, None, None, None, 1, 2, 2, 500, 96, 64, 64, 1, None) \
         == bsfa.BSFA_ERR_UNSUPPORTED
+
+
+def test_tau_table_entry_rejects_bad_arguments_without_touching_cuda(lib):
+    shape = (1, 2, 2, 500, 64, 64, 64, 1)
+    for tiles in (0, -3):
+        assert bsfa.bsfa_forward_tau_table(16, 16, 16, 16, tiles, 16, None, None, *shape, None) \
+            == bsfa.BSFA_ERR_INVALID_ARG
+        assert "tau_tiles" in bsfa.bsfa_last_error()
+    assert bsfa.bsfa_forward_tau_table(16, 16, 16, None, 4, 16, None, None, *shape, None) == bsfa.BSFA_ERR_INVALID_ARG
+    assert bsfa.bsfa_forward_tau_table(16, 16, 16, 18, 4, 16, None, None, *shape, None) == bsfa.BSFA_ERR_INVALID_ARG

@@ -1,0 +1,143 @@
+"""GPU parity for ragged sequence ends and per-position threshold tables.
+
+* Ragged ends: N that is not a multiple of the tile sizes (down to a single
+  token, and a last query tile of one row), every kernel variant, both CTA
+  pairings (two heads of a GQA group on the same rows; two adjacent tiles of one
+  head). Rows and keys past N are padding and must change nothing.
+* Per-position thresholds (§4.1, §4.2; App. B.3 "Threshold tensor"): a fixed-k
+  table [Hq, T] calibrated on other seeds, T shorter than the number of query
+  tiles so that the last column is reused; the stored c2 table at full size and,
+  calibrated at N_max = 8192, reused on the 32K layer.
+
+Comparison and tolerances are those of parity.py.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle.calibrate import calibrate, fixed_k_table
+from threshold_gated_block_b200 import bsfa
+from threshold_gated_block_b200.build import build
+from threshold_gated_block_b200.inputs import CONFIGS, custom_config, make_inputs, sample_tiles
+
+from parity import GOLDEN, all_tiles, compare_tiles, run_gpu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    build()
+    bsfa.load()
+
+
+def _inputs(N, D, Hq, Hkv, Bq, Bk, causal, kind="normal", seed=1, B=1):
+    cfg = custom_config(B=B, N=N, D=D, Hq=Hq, Hkv=Hkv, Bq=Bq, Bk=Bk, causal=causal, kind=kind, seed=seed)
+    return cfg, make_inputs(cfg)
+
+
+def _stored_table(name):
+    with open(os.path.join(GOLDEN, "tau_tables.json")) as f:
+        t = json.load(f)[name]
+    return t, np.array(t["table"], dtype=np.float64)
+
+
+# ----------------------------------------------------------------------------- ragged ends
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("Bk", [64, 128])
+@pytest.mark.parametrize("Bq", [64, 128])
+@pytest.mark.parametrize("D", [64, 128])
+def test_ragged_end_every_variant(D, Bq, Bk, causal):
+    N = 333 if causal else 461
+    cfg, x = _inputs(N, D, 4, 2, Bq, Bk, causal, seed=D + Bq + Bk + 2 * causal)
+    tau = calibrate(x["q"], x["k"], Bq, Bk, causal, [0.5])[0.5]
+    gpu = run_gpu(x, tau, Bq, Bk, causal)
+    stats = compare_tiles(x, tau, Bq, Bk, causal, gpu, all_tiles(cfg.B, cfg.Hq, N, Bq)).check()
+    assert gpu["mask"].shape == (1, 4, -(-N // Bq), -(-N // Bk))
+    assert (gpu["mask"] == 0).any() and (gpu["mask"] == 1).any()
+    print(stats)
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(4, 2), (3, 3)])
+@pytest.mark.parametrize("N", [1, 2, 63, 127, 129, 255, 257, 1000])
+@pytest.mark.parametrize("causal", [True, False])
+def test_ragged_lengths(N, Hq, Hkv, causal):
+    """Lengths around the 128-row slot and the 64-key block, for both CTA pairings;
+    at tau = +inf each row keeps only its forced blocks, so a last tile of one row
+    must still see its own key."""
+    cfg, x = _inputs(N, 128, Hq, Hkv, 128, 64, causal, kind="normal", seed=N + Hq)
+    for tau in (calibrate(x["q"], x["k"], 128, 64, causal, [0.5])[0.5], [np.inf] * Hq):
+        gpu = run_gpu(x, tau, 128, 64, causal)
+        assert np.isfinite(gpu["out"]).all() and np.isfinite(gpu["lse"]).all()
+        compare_tiles(x, tau, 128, 64, causal, gpu, all_tiles(1, Hq, N, 128)).check()
+
+
+def test_ragged_batch_keeps_sequences_apart():
+    cfg, x = _inputs(700, 64, 4, 1, 64, 128, True, kind="planted", seed=21, B=3)
+    tau = calibrate(x["q"], x["k"], 64, 128, True, [0.6])[0.6]
+    gpu = run_gpu(x, tau, 64, 128, True)
+    compare_tiles(x, tau, 64, 128, True, gpu, all_tiles(3, 4, 700, 64)).check()
+
+
+# ----------------------------------------------------------------------------- per-position threshold tables
+
+@pytest.mark.parametrize("Bq,Bk,causal", [(64, 64, True), (128, 64, True), (64, 128, False), (128, 128, False)])
+def test_fixed_k_table_small(Bq, Bk, causal):
+    """Level k = 3 of a table calibrated on two other seeds; the table stops three
+    tiles short of the sequence, so its last column serves the final tiles."""
+    N, D = 1088, 64
+    cfg, x = _inputs(N, D, 4, 2, Bq, Bk, causal, kind="planted", seed=31)
+    calib = [make_inputs(cfg, seed=s) for s in (601, 602)]
+    T = fixed_k_table([(c["q"], c["k"]) for c in calib], Bq, Bk, causal, [3])[0]
+    table = T[:, : T.shape[1] - 3].astype(np.float64)
+    gpu = run_gpu(x, table, Bq, Bk, causal)
+    stats = compare_tiles(x, table, Bq, Bk, causal, gpu, all_tiles(1, 4, N, Bq)).check()
+    assert (gpu["mask"] == 0).any() and (gpu["mask"] == 1).any()
+    print(stats)
+
+
+def test_one_column_table_is_the_per_head_threshold():
+    cfg, x = _inputs(1024, 128, 8, 2, 128, 128, True, kind="planted", seed=33)
+    tau = calibrate(x["q"], x["k"], 128, 128, True, [0.5])[0.5]
+    a = run_gpu(x, tau, 128, 128, True)
+    b = run_gpu(x, np.asarray(tau)[:, None], 128, 128, True)
+    assert np.array_equal(a["mask"], b["mask"]) and np.array_equal(a["out"], b["out"])
+    assert np.array_equal(a["lse"], b["lse"])
+
+
+@pytest.mark.parametrize("level", [0, 1, 2])
+def test_stored_table_on_the_8k_layer(level):
+    spec, T = _stored_table("c2")
+    cfg = CONFIGS["c2"]
+    x = make_inputs(cfg)
+    table = T[level]
+    gpu = run_gpu(x, table, cfg.Bq, cfg.Bk, cfg.causal)
+    stats = compare_tiles(x, table, cfg.Bq, cfg.Bk, cfg.causal, gpu, all_tiles(1, cfg.Hq, cfg.N, cfg.Bq)).check()
+    m = gpu["mask"]
+    kept = (m == 1).sum(axis=-1)
+    gated = np.isin(m, (0, 1)).sum(axis=-1)
+    k = spec["ks"][level]
+    sel = gated > k
+    stats["mean_kept_where_more_than_k"] = float(kept[sel].mean())
+    print("c2 table k =", k, stats)
+    # calibrated on other seeds: the held-out layer keeps about k blocks per tile
+    assert abs(kept[sel].mean() - k) < 0.1 * k + 1
+
+
+def test_stored_table_reused_past_its_calibrated_length():
+    """The c2 table covers 8192 tokens (64 tiles); the 32K layer's later tiles read
+    its last column (App. B.3: sequences longer than N_max reuse position N_max)."""
+    _, T = _stored_table("c2")
+    cfg = CONFIGS["c3"]
+    x = make_inputs(cfg)
+    table = T[1]
+    gpu = run_gpu(x, table, cfg.Bq, cfg.Bk, cfg.causal)
+    tiles = sample_tiles(cfg, 40)
+    assert any(i >= table.shape[1] for (_, _, i) in tiles)
+    print(compare_tiles(x, table, cfg.Bq, cfg.Bk, cfg.causal, gpu, tiles).check())

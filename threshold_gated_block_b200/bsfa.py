@@ -6,8 +6,9 @@ fallback: if the library is missing or the device is not sm_100, calls fail
 loudly.
 
 The functions named like the C entry points (``bsfa_forward``,
-``bsfa_validate``, ``bsfa_get_status``, ``bsfa_status_string``,
-``bsfa_last_error``) take the same arguments; pointer arguments accept an int
+``bsfa_forward_tau_table``, ``bsfa_validate``, ``bsfa_get_status``,
+``bsfa_selftest_lost_arrival``, ``bsfa_status_string``, ``bsfa_last_error``)
+take the same arguments; pointer arguments accept an int
 address, None, or a torch tensor (its ``data_ptr()``). ``forward`` and
 ``forward_host`` are conveniences over ``bsfa_forward`` for torch tensors.
 """
@@ -25,8 +26,8 @@ BSFA_ERR_UNSUPPORTED = 2
 BSFA_ERR_CUDA = 3
 BSFA_ERR_DEVICE_TIMEOUT = 4
 
-EXPORTED = ("bsfa_forward", "bsfa_validate", "bsfa_get_status", "bsfa_selftest_lost_arrival", "bsfa_status_string",
-            "bsfa_last_error")
+EXPORTED = ("bsfa_forward", "bsfa_forward_tau_table", "bsfa_validate", "bsfa_get_status",
+            "bsfa_selftest_lost_arrival", "bsfa_status_string", "bsfa_last_error")
 
 _lib = None
 
@@ -48,6 +49,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     vp, i = ctypes.c_void_p, ctypes.c_int
     lib.bsfa_forward.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, vp]
     lib.bsfa_forward.restype = i
+    lib.bsfa_forward_tau_table.argtypes = [vp, vp, vp, vp, i, vp, vp, vp, i, i, i, i, i, i, i, i, vp]
+    lib.bsfa_forward_tau_table.restype = i
     lib.bsfa_validate.argtypes = [i] * 8
     lib.bsfa_validate.restype = i
     lib.bsfa_get_status.argtypes = [vp]
@@ -85,6 +88,13 @@ def bsfa_forward(q, k, v, tau, out, lse, block_mask, B, Hq, Hkv, N, D, Bq, Bk, c
                                B, Hq, Hkv, N, D, Bq, Bk, int(bool(causal)), _stream(stream))
 
 
+def bsfa_forward_tau_table(q, k, v, tau_table, tau_tiles, out, lse, block_mask, B, Hq, Hkv, N, D, Bq, Bk, causal,
+                           stream) -> int:
+    return load().bsfa_forward_tau_table(_ptr(q), _ptr(k), _ptr(v), _ptr(tau_table), int(tau_tiles), _ptr(out),
+                                         _ptr(lse), _ptr(block_mask), B, Hq, Hkv, N, D, Bq, Bk, int(bool(causal)),
+                                         _stream(stream))
+
+
 def bsfa_validate(B, Hq, Hkv, N, D, Bq, Bk, causal) -> int:
     return load().bsfa_validate(B, Hq, Hkv, N, D, Bq, Bk, int(bool(causal)))
 
@@ -114,8 +124,10 @@ def _check(status: int):
 
 def forward(q, k, v, tau, *, Bq: int, Bk: int, causal: bool, want_lse: bool = True, want_mask: bool = False,
             out=None, lse=None, block_mask=None, stream=None):
-    """Run the forward on device tensors. q: bf16 [B,N,Hq,D]; k, v: bf16 [B,N,Hkv,D]; tau: fp32 [Hq].
+    """Run the forward on device tensors. q: bf16 [B,N,Hq,D]; k, v: bf16 [B,N,Hkv,D].
 
+    tau: fp32 [Hq] (one threshold per head, ``bsfa_forward``) or contiguous fp32
+    [Hq, T] (per head and query tile, ``bsfa_forward_tau_table`` with tau_tiles = T).
     Returns (out, lse or None, block_mask or None). Outputs are allocated with torch
     unless given.
     """
@@ -123,8 +135,9 @@ def forward(q, k, v, tau, *, Bq: int, Bk: int, causal: bool, want_lse: bool = Tr
     for name, t in (("q", q), ("k", k), ("v", v)):
         if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or t.dim() != 4:
             raise ValueError(f"{name} must be a contiguous 4-D bf16 CUDA tensor")
-    if tau.dtype != torch.float32 or not tau.is_cuda or tau.numel() != q.shape[2]:
-        raise ValueError("tau must be a float32 CUDA tensor with one value per query head")
+    if (tau.dtype != torch.float32 or not tau.is_cuda or not tau.is_contiguous() or tau.dim() not in (1, 2)
+            or tau.shape[0] != q.shape[2]):
+        raise ValueError("tau must be a contiguous float32 CUDA tensor [Hq] or [Hq, tiles]")
     B, N, Hq, D = q.shape
     Hkv = k.shape[2]
     if k.shape != (B, N, Hkv, D) or v.shape != k.shape:
@@ -134,18 +147,23 @@ def forward(q, k, v, tau, *, Bq: int, Bk: int, causal: bool, want_lse: bool = Tr
     if want_lse and lse is None:
         lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
     if want_mask and block_mask is None:
-        block_mask = torch.empty((B, Hq, N // Bq, N // Bk), dtype=torch.uint8, device=q.device)
+        block_mask = torch.empty((B, Hq, -(-N // Bq), -(-N // Bk)), dtype=torch.uint8, device=q.device)
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
-    _check(bsfa_forward(q, k, v, tau, out, lse if want_lse else None, block_mask if want_mask else None,
-                        B, Hq, Hkv, N, D, Bq, Bk, causal, stream))
+    lse_arg = lse if want_lse else None
+    mask_arg = block_mask if want_mask else None
+    if tau.dim() == 1:
+        _check(bsfa_forward(q, k, v, tau, out, lse_arg, mask_arg, B, Hq, Hkv, N, D, Bq, Bk, causal, stream))
+    else:
+        _check(bsfa_forward_tau_table(q, k, v, tau, tau.shape[1], out, lse_arg, mask_arg, B, Hq, Hkv, N, D, Bq, Bk,
+                                      causal, stream))
     return out, (lse if want_lse else None), (block_mask if want_mask else None)
 
 
 def forward_host(q, k, v, tau, *, Bq: int, Bk: int, causal: bool, device=None, stream=None, bufs=None):
     """End-to-end call on host tensors: copy inputs to the device, run, copy out and lse back.
 
-    q, k, v: bf16 CPU tensors (pinned for asynchronous copies); tau: fp32 CPU tensor.
+    q, k, v: bf16 CPU tensors (pinned for asynchronous copies); tau: fp32 CPU tensor, [Hq] or [Hq, T].
     ``bufs`` (from ``device_buffers``) holds reusable device and pinned host buffers.
     Returns (out_host, lse_host).
     """
@@ -154,7 +172,7 @@ def forward_host(q, k, v, tau, *, Bq: int, Bk: int, causal: bool, device=None, s
     if stream is None:
         stream = torch.cuda.current_stream(device)
     if bufs is None:
-        bufs = device_buffers(q.shape, k.shape, device)
+        bufs = device_buffers(q.shape, k.shape, device, tuple(tau.shape))
     with torch.cuda.stream(stream):
         for name, src in (("q", q), ("k", k), ("v", v), ("tau", tau)):
             bufs[name].copy_(src, non_blocking=True)
@@ -166,7 +184,7 @@ def forward_host(q, k, v, tau, *, Bq: int, Bk: int, causal: bool, device=None, s
     return bufs["out_host"], bufs["lse_host"]
 
 
-def device_buffers(q_shape, kv_shape, device):
+def device_buffers(q_shape, kv_shape, device, tau_shape=None):
     """Device inputs/outputs plus pinned host outputs for ``forward_host``."""
     import torch
     B, N, Hq, D = q_shape
@@ -174,7 +192,7 @@ def device_buffers(q_shape, kv_shape, device):
         "q": torch.empty(q_shape, dtype=torch.bfloat16, device=device),
         "k": torch.empty(kv_shape, dtype=torch.bfloat16, device=device),
         "v": torch.empty(kv_shape, dtype=torch.bfloat16, device=device),
-        "tau": torch.empty((Hq,), dtype=torch.float32, device=device),
+        "tau": torch.empty(tau_shape or (Hq,), dtype=torch.float32, device=device),
         "out": torch.empty(q_shape, dtype=torch.bfloat16, device=device),
         "lse": torch.empty((B, Hq, N), dtype=torch.float32, device=device),
         "out_host": torch.empty(q_shape, dtype=torch.bfloat16, pin_memory=True),

@@ -114,20 +114,26 @@ bsfa_status bsfa_validate(int B, int Hq, int Hkv, int N, int D, int Bq, int Bk, 
   if (D != 64 && D != 128) return fail(BSFA_ERR_UNSUPPORTED, "D=%d unsupported (64 or 128)", D);
   if ((Bq != 64 && Bq != 128) || (Bk != 64 && Bk != 128))
     return fail(BSFA_ERR_UNSUPPORTED, "Bq=%d, Bk=%d unsupported (64 or 128)", Bq, Bk);
-  if (N % 128 != 0) return fail(BSFA_ERR_UNSUPPORTED, "N=%d must be a multiple of 128", N);
-  if (N / Bk > bsfa::kMaxKeyBlocks)
-    return fail(BSFA_ERR_UNSUPPORTED, "N/Bk=%d exceeds %d key blocks", N / Bk, bsfa::kMaxKeyBlocks);
+  const int key_blocks = (int)(((long long)N + Bk - 1) / Bk);
+  if (key_blocks > bsfa::kMaxKeyBlocks)
+    return fail(BSFA_ERR_UNSUPPORTED, "ceil(N/Bk)=%d exceeds %d key blocks", key_blocks, bsfa::kMaxKeyBlocks);
   const long long rows = (long long)B * N, head_rows = (long long)B * Hq * N;
   if (rows > 0x7fffffffLL || head_rows > 0x7fffffffLL)
     return fail(BSFA_ERR_UNSUPPORTED, "B*Hq*N=%lld exceeds the 32-bit row index", head_rows);
   return BSFA_OK;
 }
 
-bsfa_status bsfa_forward(const void* q, const void* k, const void* v, const float* tau, void* out, float* lse,
-                         uint8_t* block_mask, int B, int Hq, int Hkv, int N, int D, int Bq, int Bk, int causal,
-                         void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Both entry points: tau_tiles == 0 selects one threshold per head.
+bsfa_status forward_impl(const void* q, const void* k, const void* v, const float* tau, int tau_tiles, void* out,
+                         float* lse, uint8_t* block_mask, int B, int Hq, int Hkv, int N, int D, int Bq, int Bk,
+                         int causal, void* stream) {
   bsfa_status st = bsfa_validate(B, Hq, Hkv, N, D, Bq, Bk, causal);
   if (st != BSFA_OK) return st;
+  if (tau_tiles < 0) return fail(BSFA_ERR_INVALID_ARG, "tau_tiles=%d is negative", tau_tiles);
   if (!q || !k || !v || !tau || !out) return fail(BSFA_ERR_INVALID_ARG, "q, k, v, tau and out must be non-null");
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16))
     return fail(BSFA_ERR_INVALID_ARG, "q, k, v and out must be 16-byte aligned");
@@ -142,7 +148,7 @@ bsfa_status bsfa_forward(const void* q, const void* k, const void* v, const floa
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (block_mask) {
-    const size_t n = (size_t)B * Hq * (size_t)(N / Bq) * (size_t)(N / Bk);
+    const size_t n = (size_t)B * Hq * (size_t)((N + Bq - 1) / Bq) * (size_t)((N + Bk - 1) / Bk);
     e = cudaMemsetAsync(block_mask, 3, n, s);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(block_mask)");
   }
@@ -154,6 +160,7 @@ bsfa_status bsfa_forward(const void* q, const void* k, const void* v, const floa
 
   bsfa::FwdParams p;
   p.tau = tau;
+  p.tau_tiles = tau_tiles;
   p.out = static_cast<uint16_t*>(out);
   p.lse = lse;
   p.mask = block_mask;
@@ -168,12 +175,29 @@ bsfa_status bsfa_forward(const void* q, const void* k, const void* v, const floa
   p.pair_heads = (p.group % 2 == 0) ? 1 : 0;
   p.scale = (float)(1.0 / std::sqrt((double)D));
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
-  const int tiles = N / 128;
+  const int tiles = (N + 127) / 128;
   const int grid = p.pair_heads ? B * (Hq / 2) * tiles : B * Hq * ((tiles + 1) / 2);
   e = (D == 64) ? bsfa::launch_fwd_d64(tq, tk, tv, p, Bq, Bk, causal != 0, block_mask != nullptr, grid, s)
                 : bsfa::launch_fwd_d128(tq, tk, tv, p, Bq, Bk, causal != 0, block_mask != nullptr, grid, s);
   if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
   return BSFA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+bsfa_status bsfa_forward(const void* q, const void* k, const void* v, const float* tau, void* out, float* lse,
+                         uint8_t* block_mask, int B, int Hq, int Hkv, int N, int D, int Bq, int Bk, int causal,
+                         void* stream) {
+  return forward_impl(q, k, v, tau, 0, out, lse, block_mask, B, Hq, Hkv, N, D, Bq, Bk, causal, stream);
+}
+
+bsfa_status bsfa_forward_tau_table(const void* q, const void* k, const void* v, const float* tau_table, int tau_tiles,
+                                   void* out, float* lse, uint8_t* block_mask, int B, int Hq, int Hkv, int N, int D,
+                                   int Bq, int Bk, int causal, void* stream) {
+  if (tau_tiles <= 0) return fail(BSFA_ERR_INVALID_ARG, "tau_tiles=%d must be positive", tau_tiles);
+  return forward_impl(q, k, v, tau_table, tau_tiles, out, lse, block_mask, B, Hq, Hkv, N, D, Bq, Bk, causal, stream);
 }
 
 bsfa_status bsfa_get_status(void* stream) {

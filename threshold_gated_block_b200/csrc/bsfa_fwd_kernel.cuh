@@ -3,10 +3,12 @@
 // "Block Sparse Flash Attention" (§4 Method; §4.1 Gating Mechanism; §4.4
 // Algorithm and Implementation; App. B.2 FlashAttention-2 tiled computation):
 // every score tile S_ij = Q_i K_j^T / sqrt(d) is computed exactly; the block
-// maximum s_max(i,j) is compared against the head's threshold tau; a block below
-// tau is skipped: its V tile is never loaded, its PV product is never issued and
-// the running statistics (m, l, O) are left untouched. Diagonal blocks bypass the
-// gate.
+// maximum s_max(i,j) is compared against the threshold of the head (or of the
+// head and query tile, §4.2 "Threshold Calibration"); a block below it is
+// skipped: its V tile is never loaded, its PV product is never issued and the
+// running statistics (m, l, O) are left untouched. Diagonal blocks bypass the
+// gate. N need not be a multiple of the tile sizes: query rows and keys at or
+// past N are padding (zero-filled by TMA, masked out of the gate and softmax).
 //
 // One CTA owns two 128-row query slots that read the same K/V blocks: two query
 // heads of one KV group on the same rows (GQA), or two adjacent 128-row tiles of
@@ -34,12 +36,13 @@
 namespace bsfa {
 
 struct FwdParams {
-  const float* tau;   // [Hq]
+  const float* tau;   // [Hq], or [Hq, tau_tiles] when tau_tiles > 0
+  int tau_tiles;      // 0: one threshold per head; else per (head, query tile), the last column reused past its end
   uint16_t* out;      // bf16 [B, N, Hq, D]
   float* lse;         // [B, Hq, N] or null
   uint8_t* mask;      // [B, Hq, N/Bq, N/Bk] or null
   int* status;        // device status word
-  int B, Hq, Hkv, N;
+  int B, Hq, Hkv, N;  // N need not be a multiple of the tile sizes: rows and keys >= N are masked
   int group;          // Hq / Hkv
   int pair_heads;     // 1: slots are query heads 2p and 2p+1 on the same rows
   float scale;        // 1/sqrt(D): the gate compares s_max(raw) * scale against tau
@@ -108,7 +111,7 @@ struct FwdUnit {
 };
 
 __device__ __forceinline__ FwdUnit decode_unit(const FwdParams& p, int u, bool causal, int bk) {
-  const int tiles = p.N / 128;
+  const int tiles = (p.N + 127) / 128;
   FwdUnit w;
   if (p.pair_heads) {
     // Consecutive units: the head pairs of one row block, a KV group's pairs adjacent.
@@ -133,7 +136,7 @@ __device__ __forceinline__ FwdUnit decode_unit(const FwdParams& p, int u, bool c
   w.kvh = w.hq[0] / p.group;
 #pragma unroll
   for (int s = 0; s < 2; ++s)
-    w.nblk[s] = (w.q0[s] >= p.N) ? 0 : (causal ? (w.q0[s] + 128) / bk : p.N / bk);
+    w.nblk[s] = (w.q0[s] >= p.N) ? 0 : (causal ? min((w.q0[s] + 128) / bk, (p.N + bk - 1) / bk) : (p.N + bk - 1) / bk);
   return w;
 }
 
@@ -379,11 +382,15 @@ __device__ __forceinline__ int softmax_block(const FwdParams& p, Bars* bars, uin
     else tmem_ld_x16(s_tmem + c4 * QC, raw);
 #pragma unroll
     for (int c = 0; c < QC; ++c) sv[c] = __uint_as_float(raw[c]);
+    // Last valid key of this row: the diagonal (causal) or the sequence end. A
+    // causal padding row (qrow >= N) also sees the zero-filled keys up to qrow;
+    // it is left out of the gate and never written, and V is zero there.
     const int k0 = j * BK + c4 * QC;
-    if (CAUSAL && k0 + QC - 1 > qrow) {          // this quarter reaches past the diagonal
+    const int klim = CAUSAL ? qrow : p.N - 1;
+    if (k0 + QC - 1 > klim) {                    // this thread's columns reach past it
 #pragma unroll
       for (int c = 0; c < QC; ++c)
-        if (k0 + c > qrow) sv[c] = -INFINITY;
+        if (k0 + c > klim) sv[c] = -INFINITY;
     }
     float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll
@@ -399,7 +406,7 @@ __device__ __forceinline__ int softmax_block(const FwdParams& p, Bars* bars, uin
   // A thread that must stop raises this block's abort flag before arriving, so
   // everyone reads the same value after the barrier.
   if (failed || !ok || *abort_flag) ((volatile int*)bars->sm_abort)[j & 1] = 1;
-  const bool above = ok && (pmax * p.scale >= tau);
+  const bool above = ok && qrow < p.N && (pmax * p.scale >= tau);   // rows past N are padding
   bool any_above[S::NSUB];
   any_above[0] = named_barrier_or(1, 32 * kSoftmaxWarps, above && (S::NSUB == 1 || sub == 0));
   if constexpr (S::NSUB == 2) any_above[1] = named_barrier_or(1, 32 * kSoftmaxWarps, above && sub == 1);
@@ -411,16 +418,19 @@ __device__ __forceinline__ int softmax_block(const FwdParams& p, Bars* bars, uin
   bool keep_any = false;
 #pragma unroll
   for (int t = 0; t < S::NSUB; ++t) {
-    const int lo = q0 + t * BQ, hi = lo + BQ - 1;
-    const int k_lo = j * BK, k_hi = k_lo + BK - 1;
-    const bool visible = !CAUSAL || k_lo <= hi;
-    const bool diag = CAUSAL ? (visible && k_hi > lo) : (k_lo <= hi && k_hi >= lo);
+    // Visible: some (row < N, key <= row) entry. Diagonal: judged on the full-size
+    // tile and block (as if the sequence were padded to whole tiles), so the block
+    // holding a row's own key is forced even in a last tile of one row.
+    const int lo = q0 + t * BQ;
+    const int k_lo = j * BK;
+    const bool visible = lo < p.N && (!CAUSAL || k_lo <= min(lo + BQ - 1, p.N - 1));
+    const bool diag = visible && (CAUSAL ? k_lo + BK - 1 > lo : (k_lo < lo + BQ && k_lo + BK > lo));
     code[t] = !visible ? 3 : diag ? 2 : (any_above[t] ? 1 : 0);
     keep_any |= (code[t] == 1 || code[t] == 2);
   }
   if (warp == 0 && lane == 0) {
     if (WRITE_MASK) {
-      const int mq = p.N / BQ, mkv = p.N / BK;
+      const int mq = (p.N + BQ - 1) / BQ, mkv = (p.N + BK - 1) / BK;
 #pragma unroll
       for (int t = 0; t < S::NSUB; ++t)
         if (code[t] != 3)
@@ -537,6 +547,7 @@ __device__ __forceinline__ void softmax_epilogue(const FwdParams& p, Bars* bars,
   if (!ok) return;
   tc_fence_after();
   const uint32_t o_tmem = tmem + S::TMEM_O0 + s * D + c4 * QD + ((uint32_t)(q * 32) << 16);
+  if (qrow >= p.N) return;             // padding row of the last tile
   const float inv_l = 1.f / l_row;     // > 0: every row keeps its diagonal block, which holds its own key
   uint16_t* orow = p.out + ((size_t)(w.b * p.N + qrow) * p.Hq + hq) * D + c4 * QD;
 #pragma unroll
@@ -561,7 +572,15 @@ template <int D, int BQ, int BK, bool CAUSAL, bool WRITE_MASK, typename Bars>
 __device__ __forceinline__ void softmax_role(const FwdParams& p, Bars* bars, uint32_t tmem, const FwdUnit& w) {
   SoftmaxRow<BK> st;
   bool failed = false, aborted = false;
-  const float tau0 = p.tau[w.hq[0]], tau1 = p.tau[w.hq[1]];
+  // This thread's threshold in each slot: its query tile's column of the table
+  // (clamped to the table's last column), or the head's single value.
+  const int sub = ((threadIdx.x >> 5) & 3) * 32 / BQ;
+  auto tile_tau = [&](int s) {
+    const int hq = w.hq[s];
+    const int tile = w.q0[s] / BQ + sub;
+    return p.tau_tiles > 0 ? p.tau[hq * p.tau_tiles + min(tile, p.tau_tiles - 1)] : p.tau[hq];
+  };
+  const float tau0 = tile_tau(0), tau1 = tile_tau(1);
   const int nblk = max(w.nblk[0], w.nblk[1]);
   for (int j = 0; j < nblk && !aborted; ++j) {
 #pragma unroll 1
