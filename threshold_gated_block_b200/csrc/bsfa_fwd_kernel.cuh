@@ -547,7 +547,9 @@ __device__ __forceinline__ void softmax_epilogue(const FwdParams& p, Bars* bars,
   if (!ok) return;
   tc_fence_after();
   const uint32_t o_tmem = tmem + S::TMEM_O0 + s * D + c4 * QD + ((uint32_t)(q * 32) << 16);
-  if (qrow >= p.N) return;             // padding row of the last tile
+  // Padding rows of a last tile (qrow >= N) take part in the warp's TMEM loads
+  // (warp-collective) but store nothing.
+  const bool row_ok = qrow < p.N;
   const float inv_l = 1.f / l_row;     // > 0: every row keeps its diagonal block, which holds its own key
   uint16_t* orow = p.out + ((size_t)(w.b * p.N + qrow) * p.Hq + hq) * D + c4 * QD;
 #pragma unroll
@@ -561,10 +563,12 @@ __device__ __forceinline__ void softmax_epilogue(const FwdParams& p, Bars* bars,
     for (int e = 0; e < W / 2; ++e)
       pk[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
     uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+    if (row_ok) {
 #pragma unroll
-    for (int v4 = 0; v4 < W / 8; ++v4) dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+      for (int v4 = 0; v4 < W / 8; ++v4) dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+    }
   }
-  if (c4 == 0 && p.lse != nullptr)
+  if (row_ok && c4 == 0 && p.lse != nullptr)
     p.lse[(size_t)(w.b * p.Hq + hq) * p.N + qrow] = (m + __log2f(l_row)) * 0.69314718055994531f;
 }
 
