@@ -61,6 +61,14 @@ constexpr int kLaunchRegs = kRowSplit == 2 ? 168 : 96;   // 65536 / kThreads, ro
 constexpr int kSoftmaxRegs = kRowSplit == 2 ? 216 : 104;
 constexpr int kProducerRegs = kRowSplit == 2 ? 72 : 64;
 static_assert(kSoftmaxWarps * 32 * kSoftmaxRegs + 128 * kProducerRegs <= kThreads * kLaunchRegs, "register split");
+// Named barriers: 1 = the softmax warps' gate barrier; kSReadyBar + s = "S of
+// slot s is in TMEM", which the waiter warp joins once s_full says so and the
+// softmax warps join at the start of their step (a hardware barrier, so the
+// softmax's critical path has no shared-memory poll of the MMA's completion
+// barrier).
+constexpr uint32_t kGateBar = 1;
+constexpr uint32_t kSReadyBar = 2;
+constexpr uint32_t kSReadyCount = 32 * (kSoftmaxWarps + 1);
 
 template <int D, int BQ, int BK>
 struct FwdShape {
@@ -75,7 +83,7 @@ struct FwdShape {
   static constexpr uint32_t OFF_K = OFF_Q + 2 * Q_BYTES;
   static constexpr uint32_t OFF_V = OFF_K + KS * KV_BYTES;
   static constexpr uint32_t OFF_BAR = OFF_V + VS * KV_BYTES;
-  static constexpr uint32_t BAR_BYTES = 6144;                       // barriers, gate bits, softmax exchange
+  static constexpr uint32_t BAR_BYTES = 11264;                      // barriers, gate decisions, softmax exchange
   static constexpr uint32_t SMEM_BYTES = OFF_BAR + BAR_BYTES;        // base is 1024-aligned (checked)
   static constexpr uint32_t TMEM_S0 = 0;
   static constexpr uint32_t TMEM_O0 = 2 * BK;
@@ -100,9 +108,8 @@ struct alignas(8) FwdBarriers {
   uint32_t tmem_base;
   int abort;                               // any role gave up on a bounded wait
   int sm_abort[2];                         // softmax warps' agreement to stop, by block parity
-  int decided[2];                          // blocks whose gate decision is published, per slot
-  uint32_t gate_bits[2][kMaxKeyBlocks / 32];
   float xch[2 * kRowSplit * 128];          // partial row maxima [slot][part][row]; normalisers [part][row] at the end
+  alignas(16) uint8_t gate_dec[2][kMaxKeyBlocks];   // 0 undecided, 1 skipped, 2 kept
 };
 
 struct FwdUnit {
@@ -189,13 +196,13 @@ __device__ __forceinline__ void kq_producer(const CUtensorMap* tm_q, const CUten
 // bandwidth the QK^T MMAs (both operands in shared memory) depend on.
 template <typename Bars>
 __device__ __forceinline__ bool wait_decided(Bars* bars, int s, int j) {
-  volatile int* decided = &bars->decided[s];
+  volatile uint8_t* dec = &bars->gate_dec[s][j];
   volatile int* abort_flag = &bars->abort;
-  if (*decided > j) return true;
+  if (*dec != 0) return true;
   const uint64_t t0 = global_timer_ns();
   for (;;) {
     __nanosleep(64);
-    if (*decided > j) return true;
+    if (*dec != 0) return true;
     if (*abort_flag) return false;
     if (global_timer_ns() - t0 > kWaitTimeoutNs) {
       *abort_flag = 1;
@@ -220,7 +227,7 @@ __device__ __forceinline__ void v_producer(const CUtensorMap* tm_v, uint8_t* sme
     for (int s = 0; s < 2; ++s) {
       if (j >= w.nblk[s]) continue;
       if (!wait_decided(bars, s, j)) { failed = true; break; }
-      const bool keep = (((volatile uint32_t*)bars->gate_bits[s])[j >> 5] >> (j & 31)) & 1u;
+      const bool keep = ((volatile uint8_t*)bars->gate_dec[s])[j] == 2;
       if (!keep || loaded) continue;     // skipped by this slot (or already requested)
       const int slot = v_count % S::VS;
       if (!mbar_wait(&bars->v_empty[slot], ((v_count / S::VS) & 1) ^ 1, abort_flag)) { failed = true; break; }
@@ -237,6 +244,29 @@ __device__ __forceinline__ void v_producer(const CUtensorMap* tm_v, uint8_t* sme
     drain_wait(&bars->v_full[n % S::VS], (n / S::VS) & 1);
 }
 
+// ---------------------------------------------------------------------------- S waiter (warp 11, whole warp)
+
+// Watches s_full for every (slot, block) step in the softmax warps' order and
+// joins that slot's named barrier once S is in TMEM. It syncs rather than only
+// arriving, so it stays in lockstep with the softmax warps' steps even when its
+// waits give up (then it marks the block's abort flag first and joins anyway):
+// the softmax warps never wait on a barrier that cannot complete.
+template <typename Bars>
+__device__ __forceinline__ void s_waiter(Bars* bars, const FwdUnit& w) {
+  volatile int* abort_flag = &bars->abort;
+  const int lane = threadIdx.x & 31;
+  const int nblk = max(w.nblk[0], w.nblk[1]);
+  for (int j = 0; j < nblk; ++j) {
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+      if (j >= w.nblk[s]) continue;
+      if (lane == 0 && !mbar_wait(&bars->s_full[s], j & 1, abort_flag)) ((volatile int*)bars->sm_abort)[j & 1] = 1;
+      __syncwarp();
+      named_barrier_sync(kSReadyBar + s, kSReadyCount);
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------- MMA issuer (warp 9, one thread)
 
 template <int D, int BQ, int BK, typename Bars>
@@ -245,8 +275,6 @@ __device__ __forceinline__ void mma_issuer(uint8_t* smem, Bars* bars, uint32_t t
   constexpr uint32_t IDESC_QK = make_idesc_bf16(128, BK, false);   // B = K tile, K-major
   constexpr uint32_t IDESC_PV = make_idesc_bf16(128, D, true);     // B = V tile, MN-major
   volatile int* abort_flag = &bars->abort;
-  volatile uint32_t* bits0 = bars->gate_bits[0];
-  volatile uint32_t* bits1 = bars->gate_bits[1];
   const int nblk = max(w.nblk[0], w.nblk[1]);
 
   auto qk = [&](int s, int kslot) {
@@ -294,8 +322,7 @@ __device__ __forceinline__ void mma_issuer(uint8_t* smem, Bars* bars, uint32_t t
         if (j >= w.nblk[s]) continue;
         if (!mbar_wait(&bars->p_full[s], j & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t word = s ? bits1[j >> 5] : bits0[j >> 5];
-        if ((word >> (j & 31)) & 1u) {
+        if (((volatile uint8_t*)bars->gate_dec[s])[j] == 2) {
           if (!v_ready) {
             vslot = v_count % S::VS;
             if (!mbar_wait(&bars->v_full[vslot], (v_count / S::VS) & 1, abort_flag)) { ok = false; break; }
@@ -343,9 +370,10 @@ struct SoftmaxRow {
   float l[2] = {0.f, 0.f};               // this thread's share of the running normaliser per slot
 };
 
-// Returns 2 when every softmax thread agreed to abort (a bounded wait gave up
-// somewhere), otherwise this thread's own failure flag (0 or 1), which the next
-// barrier folds into that agreement.
+// Returns 2 when the block is abandoned (a bounded wait gave up somewhere, or an
+// earlier block was abandoned: 'failed'), which every softmax thread learns
+// after the same barrier, else 0. An abandoned step still takes part in both
+// barriers, so the barrier accounting of the softmax and waiter warps agrees.
 template <int D, int BQ, int BK, bool CAUSAL, bool WRITE_MASK, typename Bars>
 __device__ __forceinline__ int softmax_block(const FwdParams& p, Bars* bars, uint32_t tmem, const FwdUnit& w,
                                              int s, int j, float tau, SoftmaxRow<BK>& st, bool failed) {
@@ -369,9 +397,10 @@ __device__ __forceinline__ int softmax_block(const FwdParams& p, Bars* bars, uin
   // before the next write to the same buffer.
   float* rowpart = &bars->xch[s * kRowSplit * 128];
 
-  bool ok = true;
-  if (lane == 0) ok = mbar_wait(&bars->s_full[s], j & 1, abort_flag);
-  ok = __shfl_sync(0xffffffffu, ok, 0);
+  // S(s, j) is in TMEM once the waiter warp has arrived (it watches s_full).
+  // After an abandoned block ('failed') the step only keeps the barriers in step.
+  named_barrier_sync(kSReadyBar + s, kSReadyCount);
+  const bool ok = !failed;
   float sv[QC];
   float pmax = -INFINITY;
   if (ok) {
@@ -403,14 +432,14 @@ __device__ __forceinline__ int softmax_block(const FwdParams& p, Bars* bars, uin
   rowpart[c4 * 128 + r] = pmax;
   // Gate: s_max * scale >= tau holds exactly when some thread's partial maximum
   // does, so the barrier's OR over the query tile's threads is the decision.
-  // A thread that must stop raises this block's abort flag before arriving, so
-  // everyone reads the same value after the barrier.
-  if (failed || !ok || *abort_flag) ((volatile int*)bars->sm_abort)[j & 1] = 1;
+  // The waiter warp raises this block's abort flag before it arrives when its
+  // wait on s_full gave up, so every softmax thread reads the same value after
+  // the gate barrier.
   const bool above = ok && qrow < p.N && (pmax * p.scale >= tau);   // rows past N are padding
   bool any_above[S::NSUB];
-  any_above[0] = named_barrier_or(1, 32 * kSoftmaxWarps, above && (S::NSUB == 1 || sub == 0));
-  if constexpr (S::NSUB == 2) any_above[1] = named_barrier_or(1, 32 * kSoftmaxWarps, above && sub == 1);
-  if (((volatile int*)bars->sm_abort)[j & 1]) return 2;
+  any_above[0] = named_barrier_or(kGateBar, 32 * kSoftmaxWarps, above && (S::NSUB == 1 || sub == 0));
+  if constexpr (S::NSUB == 2) any_above[1] = named_barrier_or(kGateBar, 32 * kSoftmaxWarps, above && sub == 1);
+  if (!ok || ((volatile int*)bars->sm_abort)[j & 1]) return 2;
   float rmax = -INFINITY;
 #pragma unroll
   for (int u = 0; u < kRowSplit; ++u) rmax = fmaxf(rmax, rowpart[u * 128 + r]);
@@ -436,16 +465,15 @@ __device__ __forceinline__ int softmax_block(const FwdParams& p, Bars* bars, uin
         if (code[t] != 3)
           p.mask[((size_t)(w.b * p.Hq + hq) * mq + (q0 / BQ + t)) * mkv + j] = (uint8_t)code[t];
     }
-    // Publish the decision (no waiting) so the V tile, if kept, is fetched right away.
-    if (keep_any) atomicOr(&bars->gate_bits[s][j >> 5], 1u << (j & 31));
-    __threadfence_block();
-    ((volatile int*)bars->decided)[s] = j + 1;
+    // Publish the decision (one byte, no fence) so the V tile, if kept, is fetched
+    // right away; the MMA warp reads it after p_full, whose arrival orders it.
+    ((volatile uint8_t*)bars->gate_dec[s])[j] = keep_any ? 2 : 1;
   }
   if (!keep_any) {                 // skipped by every tile of the slot: release S, nothing else
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(&bars->p_full[s]);
-    return failed ? 1 : 0;
+    return 0;
   }
 
   const int my_code = (S::NSUB == 1 || sub == 0) ? code[0] : code[S::NSUB - 1];
@@ -511,7 +539,7 @@ __device__ __forceinline__ int softmax_block(const FwdParams& p, Bars* bars, uin
   tc_fence_before();
   __syncwarp();
   if (lane == 0) mbar_arrive(&bars->p_full[s]);
-  return failed ? 1 : 0;
+  return 0;
 }
 
 // Epilogue of one slot: the four threads of each row combine their normalisers
@@ -575,7 +603,7 @@ __device__ __forceinline__ void softmax_epilogue(const FwdParams& p, Bars* bars,
 template <int D, int BQ, int BK, bool CAUSAL, bool WRITE_MASK, typename Bars>
 __device__ __forceinline__ void softmax_role(const FwdParams& p, Bars* bars, uint32_t tmem, const FwdUnit& w) {
   SoftmaxRow<BK> st;
-  bool failed = false, aborted = false;
+  bool aborted = false;
   // This thread's threshold in each slot: its query tile's column of the table
   // (clamped to the table's last column), or the head's single value.
   const int sub = ((threadIdx.x >> 5) & 3) * 32 / BQ;
@@ -586,19 +614,20 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, Bars* bars, uin
   };
   const float tau0 = tile_tau(0), tau1 = tile_tau(1);
   const int nblk = max(w.nblk[0], w.nblk[1]);
-  for (int j = 0; j < nblk && !aborted; ++j) {
+  // Every step is taken even after an abort (then without work), in the
+  // waiter warp's order.
+  for (int j = 0; j < nblk; ++j) {
 #pragma unroll 1
     for (int s = 0; s < 2; ++s) {
       if (j >= (s ? w.nblk[1] : w.nblk[0])) continue;
-      const int rv = softmax_block<D, BQ, BK, CAUSAL, WRITE_MASK>(p, bars, tmem, w, s, j, s ? tau1 : tau0, st, failed);
-      if (rv == 2) { aborted = true; break; }
-      failed = rv != 0;
+      if (softmax_block<D, BQ, BK, CAUSAL, WRITE_MASK>(p, bars, tmem, w, s, j, s ? tau1 : tau0, st, aborted) == 2)
+        aborted = true;
     }
   }
 #pragma unroll 1
   for (int s = 0; s < 2; ++s) {
     if ((s ? w.nblk[1] : w.nblk[0]) == 0) continue;
-    softmax_epilogue<D, BQ, BK>(p, bars, tmem, w, s, st, failed || aborted);
+    softmax_epilogue<D, BQ, BK>(p, bars, tmem, w, s, st, aborted);
   }
 }
 
@@ -626,13 +655,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->p_full[i], kSoftmaxWarps);   // one arrival per softmax warp
       mbar_init(&bars->o_done[i], 1);
       bars->sm_abort[i] = 0;
-      bars->decided[i] = 0;
     }
-    for (int i = 0; i < 2 * (kMaxKeyBlocks / 32); ++i) (&bars->gate_bits[0][0])[i] = 0u;
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
     fence_mbar_init();
   }
+  // Gate decisions start undecided (0); every thread clears a share.
+  for (int i = threadIdx.x; i < 2 * kMaxKeyBlocks / 16; i += kThreads)
+    reinterpret_cast<uint4*>(&bars->gate_dec[0][0])[i] = make_uint4(0u, 0u, 0u, 0u);
   // The 128-byte swizzle and the descriptors assume a 1024-byte aligned base.
   if ((smem_u32(smem) & 1023u) != 0) {
     if (threadIdx.x == 0) atomicOr(p.status, 2);
@@ -658,6 +688,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       else if (warp == kSoftmaxWarps + 2) v_producer<D, BQ, BK>(&tm_v, smem, bars, w);
     }
     __syncwarp();
+    if (warp == kSoftmaxWarps + 3) s_waiter(bars, w);
   }
 
   tc_fence_before();

@@ -80,6 +80,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   return mbar_wait_slow(bar, parity, abort_flag);
 }
 
+// Named barrier over `count` threads (whole warps).
+__device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t count) {
+  asm volatile("barrier.cta.sync.aligned %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // Named barrier over `count` threads that also ORs a predicate across them, so
 // every participant takes the same decision.
 __device__ __forceinline__ bool named_barrier_or(uint32_t id, uint32_t count, bool pred) {
