@@ -14,17 +14,18 @@
 // heads of one KV group on the same rows (GQA), or two adjacent 128-row tiles of
 // one head (MHA, odd group sizes). Each slot holds one query tile when Bq = 128,
 // two when Bq = 64. Warp roles (384 threads):
-//   warps 0-3, 4-7  softmax / gate / epilogue of slot 0 and slot 1: thread r of
-//                   the warpgroup owns row r of its slot (TMEM lane r);
-//   warp 8          TMEM allocation + TMA loads of both Q tiles and every K block;
-//   warp 9          tcgen05.mma issue (one thread);
-//   warp 10         TMA loads of V, issued only for blocks some slot kept;
-//   warp 11         idle (completes the producer warpgroup for the register split).
-// The two softmax warpgroups run in ping-pong: while one computes its
-// exponentials, the tensor core works on the other slot. TMEM columns: S of
-// slot 0 and 1 ([0,Bk), [Bk,2Bk)), then O of slot 0 and 1 (D columns each).
-// P is written back as bf16 over the first Bk/2 columns of its slot's S and read
-// from there as the A operand of the PV product.
+//   warps 0-7   softmax / gate / epilogue. All eight take one slot at a time and
+//               alternate slots block by block, so one slot's softmax overlaps
+//               the other slot's MMAs. Warp w owns TMEM lanes 32*(w%4)..+31 (its
+//               rows) and one half of the key columns (w/4): two threads per row.
+//   warp 8      TMEM allocation + TMA loads of both Q tiles and every K block;
+//   warp 9      tcgen05.mma issue (one thread);
+//   warp 10     TMA loads of V, issued only for blocks some slot kept;
+//   warp 11     S waiter: turns each "S is in TMEM" completion into a named
+//               barrier the softmax warps start their step on.
+// TMEM columns: S of slot 0 and 1 ([0,Bk), [Bk,2Bk)), then O of slot 0 and 1
+// (D columns each). P is written back as bf16 over the first Bk/2 columns of its
+// slot's S and read from there as the A operand of the PV product.
 //
 // MMA issue order per block j: for each slot, PV_s(j) (if kept) then QK_s(j+1).
 // The commit that announces S_s(j+1) therefore also covers PV_s(j): when the
@@ -356,7 +357,7 @@ __device__ __forceinline__ void mma_issuer(uint8_t* smem, Bars* bars, uint32_t t
   drain_wait(&bars->drain, 0);
 }
 
-// ---------------------------------------------------------------------------- softmax / gate / epilogue (warps 0-15)
+// ---------------------------------------------------------------------------- softmax / gate / epilogue (warps 0-7)
 
 // All softmax warps work on one slot at a time and alternate between the two
 // slots block by block, so a slot's softmax always overlaps the other slot's
@@ -542,8 +543,8 @@ __device__ __forceinline__ int softmax_block(const FwdParams& p, Bars* bars, uin
   return 0;
 }
 
-// Epilogue of one slot: the four threads of each row combine their normalisers
-// through shared memory, then each writes its D/4 output columns; lse is the
+// Epilogue of one slot: the two threads of each row combine their normalisers
+// through shared memory, then each writes its D/2 output columns; lse is the
 // natural-log logsumexp over the kept set.
 template <int D, int BQ, int BK, typename Bars>
 __device__ __forceinline__ void softmax_epilogue(const FwdParams& p, Bars* bars, uint32_t tmem, const FwdUnit& w,
