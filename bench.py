@@ -62,12 +62,20 @@ def parse():
                     help="gate with the stored per-position (fixed-k) table level that keeps K blocks per tile")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU-oracle baseline")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--gate", choices=["tau", "gap"], default="tau",
+                    help="tau: the BSFA gate; gap: the gap-to-running-maximum gate, for comparison")
+    ap.add_argument("--gamma", type=float, default=-1.0, help="gamma of the gap gate (scaled-score units)")
+    ap.add_argument("--curve", action="store_true",
+                    help="instead of the bench line: error against dense attention, skip fraction and time for "
+                         "several settings of each gate (one JSON line each)")
     return ap.parse_args()
 
 
 def workload(args):
     """(config, threshold description, thresholds): per head [Hq] or per position [Hq, T]."""
     cfg = CONFIGS[args.config]
+    if args.gate == "gap":
+        return cfg, {"gate": "gap to the running row maximum", "gamma": args.gamma}, [args.gamma] * cfg.Hq
     if args.tau_table is not None:
         with open(TAU_TABLES) as f:
             spec = json.load(f)[TABLE_FOR[cfg.name]]
@@ -113,14 +121,14 @@ def cpu_cores():
     return len(os.sched_getaffinity(0))
 
 
-def oracle_sample(cfg, x, taus, budget_s, tiles):
+def oracle_sample(cfg, x, taus, budget_s, tiles, gate="tau"):
     """Run the oracle on sampled tiles until the budget is spent: (dense FLOPs, seconds, tiles)."""
     from oracle import bsfa_oracle as O
     tau = np.asarray(taus, dtype=np.float64)
     f = tile_flop(cfg)
     flops, done, t0 = 0.0, 0, time.perf_counter()
     for (b, h, i) in tiles:
-        t = O.forward_tile(x["q"], x["k"], x["v"], tau, b, h, i, cfg.Bq, cfg.Bk, cfg.causal)
+        t = O.forward_tile(x["q"], x["k"], x["v"], tau, b, h, i, cfg.Bq, cfg.Bk, cfg.causal, gate=gate)
         flops += 2 * int((t["codes"] != O.CODE_INVISIBLE).sum()) * f
         done += 1
         if time.perf_counter() - t0 >= budget_s:
@@ -229,11 +237,11 @@ def run_reference(args):
     per_step = max(0.05, min(2.0, 150.0 / max(args.steps + args.warmup, 1)))
     pos = 0
     for _ in range(args.warmup):
-        _, _, n = oracle_sample(cfg, x, taus, per_step, tiles[pos:] + tiles[:pos])
+        _, _, n = oracle_sample(cfg, x, taus, per_step, tiles[pos:] + tiles[:pos], args.gate)
         pos = (pos + n) % len(tiles)
     tot_f, tot_t, tot_n = 0.0, 0.0, 0
     for _ in range(args.steps):
-        f, t, n = oracle_sample(cfg, x, taus, per_step, tiles[pos:] + tiles[:pos])
+        f, t, n = oracle_sample(cfg, x, taus, per_step, tiles[pos:] + tiles[:pos], args.gate)
         pos = (pos + n) % len(tiles)
         tot_f, tot_t, tot_n = tot_f + f, tot_t + t, tot_n + n
     value = tot_f / tot_t / 1e12
@@ -282,7 +290,10 @@ def run_ours(args):
     stream = torch.cuda.current_stream(dev)
 
     def step(t):
-        if t.dim() == 1:
+        if args.gate == "gap" and t is not tau_dense:
+            st = bsfa.bsfa_forward_gap(q, k, v, t, out, lse, None, cfg.B, cfg.Hq, cfg.Hkv, cfg.N, cfg.D, cfg.Bq, cfg.Bk,
+                                       cfg.causal, stream)
+        elif t.dim() == 1:
             st = bsfa.bsfa_forward(q, k, v, t, out, lse, None, cfg.B, cfg.Hq, cfg.Hkv, cfg.N, cfg.D, cfg.Bq, cfg.Bk,
                                    cfg.causal, stream)
         else:
@@ -292,7 +303,8 @@ def run_ours(args):
             raise RuntimeError(bsfa.bsfa_last_error())
 
     # Block codes of this layer (untimed) give the executed and dense-equivalent FLOPs.
-    _, _, mask = bsfa.forward(q, k, v, tau, Bq=cfg.Bq, Bk=cfg.Bk, causal=cfg.causal, want_lse=False, want_mask=True)
+    _, _, mask = bsfa.forward(q, k, v, tau, Bq=cfg.Bq, Bk=cfg.Bk, causal=cfg.causal, want_lse=False, want_mask=True,
+                              gate=args.gate)
     m = mask.cpu().numpy()
     del mask
     exec_flops, dense_flops = mask_flops(m, cfg)
@@ -348,7 +360,7 @@ def run_ours(args):
         ke = max(3, min(args.steps, 30))
         for _ in range(max(1, min(args.warmup, 3))):
             bsfa.forward_host(hq, hk, hv, ht, Bq=cfg.Bq, Bk=cfg.Bk, causal=cfg.causal, device=dev, stream=stream,
-                              bufs=bufs)
+                              bufs=bufs, gate=args.gate)
         barrier()
         et = []
         for _ in range(ke):
@@ -356,7 +368,7 @@ def run_ours(args):
             s1 = torch.cuda.Event(enable_timing=True)
             s0.record(stream)
             bsfa.forward_host(hq, hk, hv, ht, Bq=cfg.Bq, Bk=cfg.Bk, causal=cfg.causal, device=dev, stream=stream,
-                              bufs=bufs)
+                              bufs=bufs, gate=args.gate)
             s1.record(stream)
             torch.cuda.synchronize(dev)
             et.append(s0.elapsed_time(s1))
@@ -408,7 +420,7 @@ def run_ours(args):
             budget = args.cpu_seconds
             tiles = sample_tiles(cfg, 4096, seed=cfg.seed + 5)
             np.random.default_rng(0).shuffle(tiles)
-            f, t, n = oracle_sample(cfg, x, taus, budget, tiles)
+            f, t, n = oracle_sample(cfg, x, taus, budget, tiles, args.gate)
             line["cpu_baseline"] = {"value": f / t / 1e12, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
                                     "sample": f"{n} seeded query tiles of {cfg.name} (about {t:.1f} s of oracle "
                                               f"work), dense-equivalent FLOPs of those tiles"}
@@ -416,10 +428,86 @@ def run_ours(args):
     return 0
 
 
+# ----------------------------------------------------------------------------- gate comparison sweep
+
+GAMMA_SWEEP = (0.0, -0.25, -0.5, -0.75, -1.0, -1.5, -2.0, -3.0)
+
+
+def run_curve(args):
+    """Error against dense attention, skip fraction and kernel time for every
+    stored per-head threshold, every stored fixed-k table level and a sweep of
+    the gap gate's gamma, on one workload. The dense reference is the same
+    kernel at tau = -inf. One JSON line per setting."""
+    import torch
+    from threshold_gated_block_b200 import bsfa
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    bsfa.load()
+    cfg = CONFIGS[args.config]
+    x = make_inputs(cfg)
+    to_dev = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+    q, k, v = to_dev(x["q"]), to_dev(x["k"]), to_dev(x["v"])
+    f32 = lambda a: torch.tensor(np.asarray(a, dtype=np.float32), device=dev)
+    points = []
+    with open(TAUS) as f:
+        for p, t in sorted(json.load(f)[cfg.name]["taus"].items(), key=lambda kv: float(kv[0])):
+            points.append(("tau per head", f"target skip {p}", "tau", f32(t)))
+    if cfg.name in TABLE_FOR:
+        with open(TAU_TABLES) as f:
+            spec = json.load(f)[TABLE_FOR[cfg.name]]
+        for level, kk in enumerate(spec["ks"]):
+            points.append(("tau per position (fixed k)", f"k = {kk}", "tau", f32(spec["table"][level])))
+    for g in GAMMA_SWEEP:
+        points.append(("gap to running max", f"gamma = {g}", "gap", f32([g] * cfg.Hq)))
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def timed_ms(t, gate, reps=20):
+        run = lambda: bsfa.forward(q, k, v, t, Bq=cfg.Bq, Bk=cfg.Bk, causal=cfg.causal, want_lse=True, gate=gate,
+                                   out=out_buf, lse=lse_buf, stream=stream)
+        for _ in range(3):
+            run()
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            run()
+            e1.record(stream)
+            ts.append((e0, e1))
+        torch.cuda.synchronize(dev)
+        return float(np.median([a.elapsed_time(b) for a, b in ts]))
+
+    out_buf = torch.empty_like(q)
+    lse_buf = torch.empty((cfg.B, cfg.Hq, cfg.N), dtype=torch.float32, device=dev)
+    dense_tau = f32([float("-inf")] * cfg.Hq)
+    ref_out, ref_lse, _ = bsfa.forward(q, k, v, dense_tau, Bq=cfg.Bq, Bk=cfg.Bk, causal=cfg.causal, want_lse=True)
+    ref64 = ref_out.double()
+    ref_norm = float(ref64.norm())
+    dense_ms = timed_ms(dense_tau, "tau")
+    for (method, setting, gate, t) in points:
+        o, l, m = bsfa.forward(q, k, v, t, Bq=cfg.Bq, Bk=cfg.Bk, causal=cfg.causal, want_lse=True, want_mask=True,
+                               gate=gate)
+        mm = m.cpu().numpy()
+        gated = int(np.isin(mm, (0, 1)).sum())
+        d = o.double() - ref64
+        line = {"curve": cfg.name, "method": method, "setting": setting,
+                "skip": float((mm == 0).sum() / max(gated, 1)),
+                "out_rel_l2": float(d.norm()) / ref_norm, "out_max_abs": float(d.abs().max()),
+                "lse_mean_abs": float((l - ref_lse).abs().mean()), "ms": timed_ms(t, gate), "dense_ms": dense_ms}
+        print(json.dumps(line), flush=True)
+    if bsfa.bsfa_get_status(stream) != bsfa.BSFA_OK:
+        raise RuntimeError(bsfa.bsfa_last_error())
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.curve:
+        return run_curve(args)
     return run_ours(args)
 
 

@@ -98,6 +98,26 @@ bsfa_status bsfa_forward_tau_table(const void* q, const void* k, const void* v, 
                                    int Bq, int Bk, int causal, void* stream);
 
 /*
+ * bsfa_forward_gap - the same forward with a different gate, for comparison: the
+ * gap to the running maximum that the paper sets against its own threshold
+ * (§3 Related Work, on BLASST and SpargeAttention). The query tile visits its
+ * visible key blocks in order; each row r keeps M_r, the maximum of its scaled
+ * scores over the blocks kept so far (-inf before the first). A block that does
+ * not bypass the gate is kept when some row with a valid entry in it has a block
+ * maximum >= M_r - gamma[h]; kept blocks (diagonal ones included) then raise M_r.
+ * gamma may have either sign: a negative gamma keeps only blocks that raise
+ * some row's maximum by at least -gamma.
+ *
+ *   gamma      fp32 [Hq], device memory, in scaled-score units (q.k / sqrt(d))
+ *
+ * Every other argument, the supported set and the error behaviour are those of
+ * bsfa_forward; block_mask codes 0 and 1 record this gate's decisions.
+ */
+bsfa_status bsfa_forward_gap(const void* q, const void* k, const void* v, const float* gamma, void* out, float* lse,
+                             uint8_t* block_mask, int B, int Hq, int Hkv, int N, int D, int Bq, int Bk, int causal,
+                             void* stream);
+
+/*
  * bsfa_validate - the shape checks of bsfa_forward, host only (no CUDA call).
  * Returns BSFA_OK, BSFA_ERR_INVALID_ARG or BSFA_ERR_UNSUPPORTED.
  */

@@ -94,3 +94,59 @@ def brute_forward(q, k, v, tau, Bq: int, Bk: int, causal: bool):
                     out[b][r][hq][d] = sum(w * v[b][c][g][d] for w, c in zip(weights, kept)) / total
                 lse[b][hq][r] = m + math.log(total)
     return out, lse, codes
+
+
+def brute_gap_codes(q, k, gamma, Bq: int, Bk: int, causal: bool):
+    """Block codes under the gap-to-running-maximum gate, by plain loops.
+
+    For each query tile the visible key blocks are visited in increasing order.
+    Row r's running maximum starts at -inf and takes in every score of every kept
+    block. A block that is not forced is kept when some row with a valid entry in
+    it has no kept block yet or reaches at least (running maximum - gamma[hq]). Forced and visible blocks
+    are found by enumerating the full-size tile and block, as in ``brute_forward``.
+    Returns {(b, hq, i, j): code}.
+    """
+    B, N, Hq, D = len(q), len(q[0]), len(q[0][0]), len(q[0][0][0])
+    Hkv = len(k[0][0])
+    per_kv = Hq // Hkv
+    inv = 1.0 / math.sqrt(D)
+    mq = (N + Bq - 1) // Bq
+    mkv = (N + Bk - 1) // Bk
+    codes = {}
+    for b in range(B):
+        for hq in range(Hq):
+            g = hq // per_kv
+            for i in range(mq):
+                rows = list(range(i * Bq, min((i + 1) * Bq, N)))
+                run = {r: -math.inf for r in rows}
+                for j in range(mkv):
+                    cols = list(range(j * Bk, min((j + 1) * Bk, N)))
+                    best = {}
+                    for r in rows:
+                        for c in cols:
+                            if _is_valid(r, c, causal):
+                                acc = 0.0
+                                for d in range(D):
+                                    acc += q[b][r][hq][d] * k[b][c][g][d]
+                                val = acc * inv
+                                if r not in best or val > best[r]:
+                                    best[r] = val
+                    if not best:
+                        codes[(b, hq, i, j)] = 3
+                        continue
+                    full_rows = range(i * Bq, (i + 1) * Bq)
+                    full_cols = range(j * Bk, (j + 1) * Bk)
+                    if causal:
+                        forced = any(not _is_valid(r, c, True) for r in full_rows for c in full_cols)
+                    else:
+                        forced = any(c in full_rows for c in full_cols)
+                    if forced:
+                        code = 2
+                    else:
+                        code = 1 if any(run[r] == -math.inf or best[r] >= run[r] - gamma[hq] for r in best) else 0
+                    codes[(b, hq, i, j)] = code
+                    if code != 0:
+                        for r, val in best.items():
+                            if val > run[r]:
+                                run[r] = val
+    return codes

@@ -46,6 +46,18 @@ design notes):
 
 Block codes: 0 = skipped by the gate, 1 = kept by the gate, 2 = forced keep
 (diagonal), 3 = not visible (causally masked out entirely).
+
+A second gate is provided for comparison (``gate="gap"``): the gap to the
+running maximum, which the page attributes to BLASST and SpargeAttention (§3
+Related Work, paragraphs "Gating after scoring" and "Predicting importance
+before scoring"): a block is skipped when it lies far below the running maximum. The
+pages give no formula, so the reading here is: the query tile visits its
+visible key blocks in increasing order; each row r keeps M_r, the maximum of
+its scores over the blocks kept so far (-inf at first); a non-diagonal block
+is kept when some row with a valid entry in it has no kept block yet or has
+rowmax_r(block) >= M_r - gamma (gamma per head, in scaled-score units, of either
+sign); kept blocks (diagonal ones included) then raise M_r. Skipped blocks leave M_r alone, as they leave
+the softmax statistics alone in BSFA.
 """
 from __future__ import annotations
 
@@ -174,6 +186,43 @@ def tile_block_codes(S: np.ndarray, valid: np.ndarray, i: int, tau: float, Bq: i
     return codes, smax
 
 
+def tile_block_codes_gap(S: np.ndarray, valid: np.ndarray, i: int, gamma: float, Bq: int, Bk: int,
+                         N: int, causal: bool, flip=()) -> tuple[np.ndarray, np.ndarray]:
+    """Block codes of one query tile under the gap-to-running-maximum gate.
+
+    Returns (codes, margin): margin[j] is, for a gated block, the largest over its
+    rows with a valid entry of rowmax_r - (M_r - gamma) (kept iff >= 0); NaN for
+    forced and invisible blocks. ``flip`` inverts the decision of the named gated
+    blocks, and later blocks follow the flipped running maxima.
+    """
+    mkv = -(-N // Bk)
+    codes = np.full(mkv, CODE_INVISIBLE, dtype=np.uint8)
+    margin = np.full(mkv, np.nan)
+    ncols = S.shape[1]
+    M = np.full(S.shape[0], -np.inf)
+    for j in range(mkv):
+        if not block_visible(i, j, Bq, Bk, N, causal):
+            continue
+        c0, c1 = j * Bk, min((j + 1) * Bk, ncols)
+        blk = np.where(valid[:, c0:c1], S[:, c0:c1], -np.inf) if c0 < ncols else np.full((S.shape[0], 1), -np.inf)
+        rowmax = blk.max(axis=1)
+        if block_diagonal(i, j, Bq, Bk, N, causal):
+            codes[j] = CODE_FORCED
+        else:
+            part = np.isfinite(rowmax)
+            # a row with no kept block yet (M = -inf) always qualifies
+            with np.errstate(invalid="ignore"):      # -inf - (-inf) in the branch not taken
+                gaps = np.where(np.isneginf(M[part]), np.inf, rowmax[part] - (M[part] - gamma))
+            margin[j] = float(gaps.max()) if gaps.size else -np.inf
+            keep = bool(gaps.size) and margin[j] >= 0.0
+            if j in flip:
+                keep = not keep
+            codes[j] = CODE_KEPT if keep else CODE_SKIPPED
+        if codes[j] in (CODE_KEPT, CODE_FORCED):
+            M = np.maximum(M, rowmax)
+    return codes, margin
+
+
 def tile_softmax(S: np.ndarray, valid: np.ndarray, codes: np.ndarray, vmat: np.ndarray,
                  Bk: int) -> tuple[np.ndarray, np.ndarray]:
     """Softmax over the kept key set only (§4.4: skipped blocks never enter m, l, O)."""
@@ -191,7 +240,7 @@ def tile_softmax(S: np.ndarray, valid: np.ndarray, codes: np.ndarray, vmat: np.n
 
 
 def forward_tile(q_bits, k_bits, v_bits, tau, b: int, hq: int, i: int, Bq: int, Bk: int,
-                 causal: bool, flip=(), with_output: bool = True) -> dict:
+                 causal: bool, flip=(), with_output: bool = True, gate: str = "tau") -> dict:
     """The BSFA result for one query tile (b, hq, i).
 
     q_bits: uint16 [B, N, Hq, D]; k_bits, v_bits: uint16 [B, N, Hkv, D]; tau: [Hq] or [Hq, M]
@@ -207,16 +256,24 @@ def forward_tile(q_bits, k_bits, v_bits, tau, b: int, hq: int, i: int, Bq: int, 
     kmat = widen_bf16(k_bits[b, :ncols, g, :])
     S = tile_scores(qi, kmat, D)
     valid = valid_mask(r0, r1, ncols, causal)
-    codes, smax = tile_block_codes(S, valid, i, tile_tau(tau, hq, i), Bq, Bk, N, causal, flip)
-    res = {"codes": codes, "smax": smax, "rows": (r0, r1)}
+    if gate == "gap":
+        codes, margin = tile_block_codes_gap(S, valid, i, tile_tau(tau, hq, i), Bq, Bk, N, causal, flip)
+        res = {"codes": codes, "margin": margin, "rows": (r0, r1)}
+    else:
+        codes, smax = tile_block_codes(S, valid, i, tile_tau(tau, hq, i), Bq, Bk, N, causal, flip)
+        res = {"codes": codes, "smax": smax, "rows": (r0, r1)}
     if with_output:
         vmat = widen_bf16(v_bits[b, :ncols, g, :])
         res["out"], res["lse"] = tile_softmax(S, valid, codes, vmat, Bk)
     return res
 
 
-def forward(q_bits, k_bits, v_bits, tau, Bq: int, Bk: int, causal: bool) -> dict:
-    """The whole BSFA forward: out [B,N,Hq,D], lse [B,Hq,N], codes/smax [B,Hq,M_Q,M_KV]."""
+def forward(q_bits, k_bits, v_bits, tau, Bq: int, Bk: int, causal: bool, gate: str = "tau") -> dict:
+    """The whole BSFA forward: out [B,N,Hq,D], lse [B,Hq,N], codes/smax [B,Hq,M_Q,M_KV].
+
+    gate="gap" uses the gap-to-running-maximum gate with ``tau`` holding gamma;
+    "smax" then holds each gated block's margin instead.
+    """
     B, N, Hq, D = q_bits.shape
     mq, mkv = -(-N // Bq), -(-N // Bk)
     out = np.zeros((B, N, Hq, D))
@@ -227,12 +284,12 @@ def forward(q_bits, k_bits, v_bits, tau, Bq: int, Bk: int, causal: bool) -> dict
     for b in range(B):
         for hq in range(Hq):
             for i in range(mq):
-                t = forward_tile(q_bits, k_bits, v_bits, tau, b, hq, i, Bq, Bk, causal)
+                t = forward_tile(q_bits, k_bits, v_bits, tau, b, hq, i, Bq, Bk, causal, gate=gate)
                 r0, r1 = t["rows"]
                 out[b, r0:r1, hq, :] = t["out"]
                 lse[b, hq, r0:r1] = t["lse"]
                 codes[b, hq, i] = t["codes"]
-                smax[b, hq, i] = t["smax"]
+                smax[b, hq, i] = t["margin" if gate == "gap" else "smax"]
     return {"out": out, "lse": lse, "codes": codes, "smax": smax}
 
 

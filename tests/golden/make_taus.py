@@ -21,6 +21,9 @@ from oracle.calibrate import calibrate  # noqa: E402
 
 OUT = os.path.join(HERE, "taus.json")
 
+# Extra skip targets beyond a workload's own, for the gate comparison sweep.
+EXTRA_SKIPS = {"c2": (0.3, 0.7, 0.9)}
+
 
 def main(names):
     table = {}
@@ -32,7 +35,8 @@ def main(names):
         t0 = time.time()
         x = make_inputs(cfg)
         tiles = sample_tiles(cfg, cfg.sampled_tiles) if cfg.sampled_tiles else None
-        taus = calibrate(x["q"], x["k"], cfg.Bq, cfg.Bk, cfg.causal, cfg.skips, tiles)
+        skips = tuple(sorted(set(cfg.skips) | set(EXTRA_SKIPS.get(name, ()))))
+        taus = calibrate(x["q"], x["k"], cfg.Bq, cfg.Bk, cfg.causal, skips, tiles)
         table[name] = {
             "taus": {str(p): t for p, t in taus.items()},
             "calibrated_on": "sampled tiles" if tiles else "all tiles",

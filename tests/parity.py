@@ -37,10 +37,11 @@ def to_device(bits: np.ndarray) -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
 
 
-def run_gpu(x: dict, tau, Bq: int, Bk: int, causal: bool, want_mask: bool = True):
+def run_gpu(x: dict, tau, Bq: int, Bk: int, causal: bool, want_mask: bool = True, gate: str = "tau"):
     q, k, v = (to_device(x[n]) for n in "qkv")
     t = torch.tensor(np.asarray(tau, dtype=np.float32), device="cuda")
-    out, lse, mask = bsfa.forward(q, k, v, t, Bq=Bq, Bk=Bk, causal=causal, want_lse=True, want_mask=want_mask)
+    out, lse, mask = bsfa.forward(q, k, v, t, Bq=Bq, Bk=Bk, causal=causal, want_lse=True, want_mask=want_mask,
+                                  gate=gate)
     torch.cuda.synchronize()
     assert bsfa.bsfa_get_status(None) == bsfa.BSFA_OK, bsfa.bsfa_last_error()
     res = {
@@ -74,25 +75,32 @@ class Report:
                 "near_tau": self.near_tau, "flipped": self.flipped}
 
 
-def compare_tiles(x: dict, tau, Bq: int, Bk: int, causal: bool, gpu: dict, tiles, report: Report | None = None):
-    """Compare the GPU result with the oracle on the given (b, hq, i) tiles."""
+def compare_tiles(x: dict, tau, Bq: int, Bk: int, causal: bool, gpu: dict, tiles, report: Report | None = None,
+                  gate: str = "tau"):
+    """Compare the GPU result with the oracle on the given (b, hq, i) tiles.
+
+    gate="gap": the gap gate with tau holding gamma; a gated block is near the
+    boundary when its margin (largest row excess over M_r - gamma) is within
+    NEAR_TAU of zero.
+    """
     rep = report or Report()
     tau = np.asarray(tau, dtype=np.float64)
     for (b, hq, i) in tiles:
         tau_i = O.tile_tau(tau, hq, i)
-        t = O.forward_tile(x["q"], x["k"], x["v"], tau, b, hq, i, Bq, Bk, causal)
+        t = O.forward_tile(x["q"], x["k"], x["v"], tau, b, hq, i, Bq, Bk, causal, gate=gate)
         flip = ()
         if gpu["mask"] is not None:
             gm = gpu["mask"][b, hq, i]
             gated = np.isin(t["codes"], (O.CODE_SKIPPED, O.CODE_KEPT))
-            near = gated & (np.abs(t["smax"] - tau_i) <= NEAR_TAU)
+            dist = np.abs(t["margin"]) if gate == "gap" else np.abs(t["smax"] - tau_i)
+            near = gated & (dist <= NEAR_TAU)
             rep.near_tau += int(near.sum())
             differ = gm != t["codes"]
             flip = tuple(int(j) for j in np.nonzero(differ & near)[0])
             rep.mask_mismatch += int((differ & ~near).sum())
             if flip:
                 rep.flipped += len(flip)
-                t = O.forward_tile(x["q"], x["k"], x["v"], tau, b, hq, i, Bq, Bk, causal, flip=flip)
+                t = O.forward_tile(x["q"], x["k"], x["v"], tau, b, hq, i, Bq, Bk, causal, flip=flip, gate=gate)
         r0, r1 = t["rows"]
         d = np.abs(gpu["out"][b, r0:r1, hq, :] - t["out"])
         rep.max_abs = max(rep.max_abs, float(d.max()))

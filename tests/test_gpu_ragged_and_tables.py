@@ -8,6 +8,9 @@
   table [Hq, T] calibrated on other seeds, T shorter than the number of query
   tiles so that the last column is reused; the stored c2 table at full size and,
   calibrated at N_max = 8192, reused on the 32K layer.
+* The gap-to-running-maximum gate (bsfa_forward_gap), with gammas chosen so no
+  compared block sits within 1e-3 of the gate's boundary (its decisions cascade
+  through the running maxima, so a near tie is avoided rather than flipped).
 
 Comparison and tolerances are those of parity.py.
 """
@@ -141,3 +144,48 @@ def test_stored_table_reused_past_its_calibrated_length():
     tiles = sample_tiles(cfg, 40)
     assert any(i >= table.shape[1] for (_, _, i) in tiles)
     print(compare_tiles(x, table, cfg.Bq, cfg.Bk, cfg.causal, gpu, tiles).check())
+
+
+# ----------------------------------------------------------------------------- the gap gate (comparison)
+
+def _gap_gammas(x, Hq, Bq, Bk, causal, base, tiles):
+    """One gamma per head near ``base``, nudged until no gated block of the
+    compared tiles lies within 10x the near band of the gate's boundary."""
+    from oracle import bsfa_oracle as O
+    gam = [base + 0.037 * h for h in range(Hq)]
+    for _ in range(8):
+        near = False
+        for (b, hq, i) in tiles:
+            t = O.forward_tile(x["q"], x["k"], None, gam, b, hq, i, Bq, Bk, causal, with_output=False, gate="gap")
+            m = t["margin"][np.isfinite(t["margin"])]
+            if (np.abs(m) <= 1e-3).any():
+                gam[hq] += 0.0123
+                near = True
+        if not near:
+            return gam
+    return gam
+
+
+@pytest.mark.parametrize("Bq,Bk,causal,N", [(128, 128, True, 1024), (64, 64, True, 700), (128, 64, False, 768),
+                                              (64, 128, False, 640)])
+def test_gap_gate_small(Bq, Bk, causal, N):
+    cfg, x = _inputs(N, 64, 4, 2, Bq, Bk, causal, kind="planted", seed=50 + Bq + Bk)
+    tiles = all_tiles(1, 4, N, Bq)
+    gam = _gap_gammas(x, 4, Bq, Bk, causal, -0.8, tiles)
+    gpu = run_gpu(x, gam, Bq, Bk, causal, gate="gap")
+    stats = compare_tiles(x, gam, Bq, Bk, causal, gpu, tiles, gate="gap").check()
+    assert (gpu["mask"] == 0).any() and (gpu["mask"] == 1).any()
+    print(stats)
+
+
+def test_gap_gate_on_the_8k_layer():
+    cfg = CONFIGS["c2"]
+    x = make_inputs(cfg)
+    tiles = sample_tiles(cfg, 48)
+    gam = _gap_gammas(x, cfg.Hq, cfg.Bq, cfg.Bk, cfg.causal, -1.0, tiles)
+    gpu = run_gpu(x, gam, cfg.Bq, cfg.Bk, cfg.causal, gate="gap")
+    stats = compare_tiles(x, gam, cfg.Bq, cfg.Bk, cfg.causal, gpu, tiles, gate="gap").check()
+    m = gpu["mask"]
+    stats["skip_fraction"] = float((m == 0).sum() / max(np.isin(m, (0, 1)).sum(), 1))
+    print("c2 gap", stats)
+    assert 0.2 < stats["skip_fraction"] < 0.95

@@ -6,7 +6,7 @@ fallback: if the library is missing or the device is not sm_100, calls fail
 loudly.
 
 The functions named like the C entry points (``bsfa_forward``,
-``bsfa_forward_tau_table``, ``bsfa_validate``, ``bsfa_get_status``,
+``bsfa_forward_tau_table``, ``bsfa_forward_gap``, ``bsfa_validate``, ``bsfa_get_status``,
 ``bsfa_selftest_lost_arrival``, ``bsfa_status_string``, ``bsfa_last_error``)
 take the same arguments; pointer arguments accept an int
 address, None, or a torch tensor (its ``data_ptr()``). ``forward`` and
@@ -26,7 +26,7 @@ BSFA_ERR_UNSUPPORTED = 2
 BSFA_ERR_CUDA = 3
 BSFA_ERR_DEVICE_TIMEOUT = 4
 
-EXPORTED = ("bsfa_forward", "bsfa_forward_tau_table", "bsfa_validate", "bsfa_get_status",
+EXPORTED = ("bsfa_forward", "bsfa_forward_tau_table", "bsfa_forward_gap", "bsfa_validate", "bsfa_get_status",
             "bsfa_selftest_lost_arrival", "bsfa_status_string", "bsfa_last_error")
 
 _lib = None
@@ -51,6 +51,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.bsfa_forward.restype = i
     lib.bsfa_forward_tau_table.argtypes = [vp, vp, vp, vp, i, vp, vp, vp, i, i, i, i, i, i, i, i, vp]
     lib.bsfa_forward_tau_table.restype = i
+    lib.bsfa_forward_gap.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, vp]
+    lib.bsfa_forward_gap.restype = i
     lib.bsfa_validate.argtypes = [i] * 8
     lib.bsfa_validate.restype = i
     lib.bsfa_get_status.argtypes = [vp]
@@ -95,6 +97,11 @@ def bsfa_forward_tau_table(q, k, v, tau_table, tau_tiles, out, lse, block_mask, 
                                          _stream(stream))
 
 
+def bsfa_forward_gap(q, k, v, gamma, out, lse, block_mask, B, Hq, Hkv, N, D, Bq, Bk, causal, stream) -> int:
+    return load().bsfa_forward_gap(_ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(out), _ptr(lse), _ptr(block_mask),
+                                   B, Hq, Hkv, N, D, Bq, Bk, int(bool(causal)), _stream(stream))
+
+
 def bsfa_validate(B, Hq, Hkv, N, D, Bq, Bk, causal) -> int:
     return load().bsfa_validate(B, Hq, Hkv, N, D, Bq, Bk, int(bool(causal)))
 
@@ -123,11 +130,12 @@ def _check(status: int):
 
 
 def forward(q, k, v, tau, *, Bq: int, Bk: int, causal: bool, want_lse: bool = True, want_mask: bool = False,
-            out=None, lse=None, block_mask=None, stream=None):
+            out=None, lse=None, block_mask=None, stream=None, gate: str = "tau"):
     """Run the forward on device tensors. q: bf16 [B,N,Hq,D]; k, v: bf16 [B,N,Hkv,D].
 
     tau: fp32 [Hq] (one threshold per head, ``bsfa_forward``) or contiguous fp32
     [Hq, T] (per head and query tile, ``bsfa_forward_tau_table`` with tau_tiles = T).
+    gate="gap": ``bsfa_forward_gap`` with tau holding gamma [Hq].
     Returns (out, lse or None, block_mask or None). Outputs are allocated with torch
     unless given.
     """
@@ -152,7 +160,11 @@ def forward(q, k, v, tau, *, Bq: int, Bk: int, causal: bool, want_lse: bool = Tr
         stream = torch.cuda.current_stream(q.device)
     lse_arg = lse if want_lse else None
     mask_arg = block_mask if want_mask else None
-    if tau.dim() == 1:
+    if gate == "gap":
+        if tau.dim() != 1:
+            raise ValueError("the gap gate takes one gamma per head")
+        _check(bsfa_forward_gap(q, k, v, tau, out, lse_arg, mask_arg, B, Hq, Hkv, N, D, Bq, Bk, causal, stream))
+    elif tau.dim() == 1:
         _check(bsfa_forward(q, k, v, tau, out, lse_arg, mask_arg, B, Hq, Hkv, N, D, Bq, Bk, causal, stream))
     else:
         _check(bsfa_forward_tau_table(q, k, v, tau, tau.shape[1], out, lse_arg, mask_arg, B, Hq, Hkv, N, D, Bq, Bk,
@@ -160,7 +172,8 @@ def forward(q, k, v, tau, *, Bq: int, Bk: int, causal: bool, want_lse: bool = Tr
     return out, (lse if want_lse else None), (block_mask if want_mask else None)
 
 
-def forward_host(q, k, v, tau, *, Bq: int, Bk: int, causal: bool, device=None, stream=None, bufs=None):
+def forward_host(q, k, v, tau, *, Bq: int, Bk: int, causal: bool, device=None, stream=None, bufs=None,
+                 gate: str = "tau"):
     """End-to-end call on host tensors: copy inputs to the device, run, copy out and lse back.
 
     q, k, v: bf16 CPU tensors (pinned for asynchronous copies); tau: fp32 CPU tensor, [Hq] or [Hq, T].
@@ -177,7 +190,7 @@ def forward_host(q, k, v, tau, *, Bq: int, Bk: int, causal: bool, device=None, s
         for name, src in (("q", q), ("k", k), ("v", v), ("tau", tau)):
             bufs[name].copy_(src, non_blocking=True)
         forward(bufs["q"], bufs["k"], bufs["v"], bufs["tau"], Bq=Bq, Bk=Bk, causal=causal, out=bufs["out"],
-                lse=bufs["lse"], stream=stream)
+                lse=bufs["lse"], stream=stream, gate=gate)
         bufs["out_host"].copy_(bufs["out"], non_blocking=True)
         bufs["lse_host"].copy_(bufs["lse"], non_blocking=True)
     stream.synchronize()

@@ -127,10 +127,11 @@ bsfa_status bsfa_validate(int B, int Hq, int Hkv, int N, int D, int Bq, int Bk, 
 
 namespace {
 
-// Both entry points: tau_tiles == 0 selects one threshold per head.
-bsfa_status forward_impl(const void* q, const void* k, const void* v, const float* tau, int tau_tiles, void* out,
-                         float* lse, uint8_t* block_mask, int B, int Hq, int Hkv, int N, int D, int Bq, int Bk,
-                         int causal, void* stream) {
+// Every forward entry point: tau_tiles == 0 selects one value per head; gate_gap
+// selects the gap gate, tau then holding gamma.
+bsfa_status forward_impl(const void* q, const void* k, const void* v, const float* tau, int tau_tiles, int gate_gap,
+                         void* out, float* lse, uint8_t* block_mask, int B, int Hq, int Hkv, int N, int D, int Bq,
+                         int Bk, int causal, void* stream) {
   bsfa_status st = bsfa_validate(B, Hq, Hkv, N, D, Bq, Bk, causal);
   if (st != BSFA_OK) return st;
   if (tau_tiles < 0) return fail(BSFA_ERR_INVALID_ARG, "tau_tiles=%d is negative", tau_tiles);
@@ -161,6 +162,7 @@ bsfa_status forward_impl(const void* q, const void* k, const void* v, const floa
   bsfa::FwdParams p;
   p.tau = tau;
   p.tau_tiles = tau_tiles;
+  p.gate_gap = gate_gap;
   p.out = static_cast<uint16_t*>(out);
   p.lse = lse;
   p.mask = block_mask;
@@ -190,14 +192,21 @@ extern "C" {
 bsfa_status bsfa_forward(const void* q, const void* k, const void* v, const float* tau, void* out, float* lse,
                          uint8_t* block_mask, int B, int Hq, int Hkv, int N, int D, int Bq, int Bk, int causal,
                          void* stream) {
-  return forward_impl(q, k, v, tau, 0, out, lse, block_mask, B, Hq, Hkv, N, D, Bq, Bk, causal, stream);
+  return forward_impl(q, k, v, tau, 0, 0, out, lse, block_mask, B, Hq, Hkv, N, D, Bq, Bk, causal, stream);
 }
 
 bsfa_status bsfa_forward_tau_table(const void* q, const void* k, const void* v, const float* tau_table, int tau_tiles,
                                    void* out, float* lse, uint8_t* block_mask, int B, int Hq, int Hkv, int N, int D,
                                    int Bq, int Bk, int causal, void* stream) {
   if (tau_tiles <= 0) return fail(BSFA_ERR_INVALID_ARG, "tau_tiles=%d must be positive", tau_tiles);
-  return forward_impl(q, k, v, tau_table, tau_tiles, out, lse, block_mask, B, Hq, Hkv, N, D, Bq, Bk, causal, stream);
+  return forward_impl(q, k, v, tau_table, tau_tiles, 0, out, lse, block_mask, B, Hq, Hkv, N, D, Bq, Bk, causal,
+                      stream);
+}
+
+bsfa_status bsfa_forward_gap(const void* q, const void* k, const void* v, const float* gamma, void* out, float* lse,
+                             uint8_t* block_mask, int B, int Hq, int Hkv, int N, int D, int Bq, int Bk, int causal,
+                             void* stream) {
+  return forward_impl(q, k, v, gamma, 0, 1, out, lse, block_mask, B, Hq, Hkv, N, D, Bq, Bk, causal, stream);
 }
 
 bsfa_status bsfa_get_status(void* stream) {

@@ -46,6 +46,7 @@ struct FwdParams {
   int B, Hq, Hkv, N;  // N need not be a multiple of the tile sizes: rows and keys >= N are masked
   int group;          // Hq / Hkv
   int pair_heads;     // 1: slots are query heads 2p and 2p+1 on the same rows
+  int gate_gap;       // 0: the BSFA gate (block maximum against tau); 1: the gap gate, tau holding gamma
   float scale;        // 1/sqrt(D): the gate compares s_max(raw) * scale against tau
   float scale_log2;   // log2(e)/sqrt(D): exponent scale of the softmax
 };
@@ -367,8 +368,9 @@ __device__ __forceinline__ void mma_issuer(uint8_t* smem, Bars* bars, uint32_t t
 // the block's named barrier computes over the threads' own comparisons.
 template <int BK>
 struct SoftmaxRow {
-  float m[2] = {-INFINITY, -INFINITY};   // running row maximum per slot, exp2 domain
+  float m[2] = {-INFINITY, -INFINITY};   // reference maximum of the exponentials per slot, exp2 domain (lazy)
   float l[2] = {0.f, 0.f};               // this thread's share of the running normaliser per slot
+  float M[2] = {-INFINITY, -INFINITY};   // true row maximum over the kept blocks per slot, exp2 domain (gap gate)
 };
 
 // Returns 2 when the block is abandoned (a bounded wait gave up somewhere, or an
@@ -436,7 +438,14 @@ __device__ __forceinline__ int softmax_block(const FwdParams& p, Bars* bars, uin
   // The waiter warp raises this block's abort flag before it arrives when its
   // wait on s_full gave up, so every softmax thread reads the same value after
   // the gate barrier.
-  const bool above = ok && qrow < p.N && (pmax * p.scale >= tau);   // rows past N are padding
+  // Rows past N are padding. The gap gate (tau = gamma * log2(e)) keeps the block
+  // when some row with a valid entry has no kept block yet or reaches its running
+  // maximum minus gamma.
+  const float run_max = s ? st.M[1] : st.M[0];
+  const bool above =
+      ok && qrow < p.N &&
+      (p.gate_gap ? (pmax > -INFINITY && (run_max == -INFINITY || pmax * p.scale_log2 >= run_max - tau))
+                  : (pmax * p.scale >= tau));
   bool any_above[S::NSUB];
   any_above[0] = named_barrier_or(kGateBar, 32 * kSoftmaxWarps, above && (S::NSUB == 1 || sub == 0));
   if constexpr (S::NSUB == 2) any_above[1] = named_barrier_or(kGateBar, 32 * kSoftmaxWarps, above && sub == 1);
@@ -485,6 +494,7 @@ __device__ __forceinline__ int softmax_block(const FwdParams& p, Bars* bars, uin
   float alpha = 1.f;
   if (my_keep) {
     const float mx = rmax * p.scale_log2;
+    if (s) st.M[1] = fmaxf(st.M[1], mx); else st.M[0] = fmaxf(st.M[0], mx);
     if (mx > m + kRescaleThreshold) {      // also taken on the first finite maximum
       if (m != -INFINITY) {
         alpha = ex2_approx(m - mx);
@@ -611,7 +621,8 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, Bars* bars, uin
   auto tile_tau = [&](int s) {
     const int hq = w.hq[s];
     const int tile = w.q0[s] / BQ + sub;
-    return p.tau_tiles > 0 ? p.tau[hq * p.tau_tiles + min(tile, p.tau_tiles - 1)] : p.tau[hq];
+    const float t = p.tau_tiles > 0 ? p.tau[hq * p.tau_tiles + min(tile, p.tau_tiles - 1)] : p.tau[hq];
+    return p.gate_gap ? t * 1.4426950408889634f : t;   // gamma in the exp2 domain of the running maximum
   };
   const float tau0 = tile_tau(0), tau1 = tile_tau(1);
   const int nblk = max(w.nblk[0], w.nblk[1]);
