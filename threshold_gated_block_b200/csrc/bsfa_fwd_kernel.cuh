@@ -47,6 +47,7 @@ struct FwdParams {
   int group;          // Hq / Hkv
   int pair_heads;     // 1: slots are query heads 2p and 2p+1 on the same rows
   int gate_gap;       // 0: the BSFA gate (block maximum against tau); 1: the gap gate, tau holding gamma
+                      // (selects the kernel's GAP template argument at launch)
   float scale;        // 1/sqrt(D): the gate compares s_max(raw) * scale against tau
   float scale_log2;   // log2(e)/sqrt(D): exponent scale of the softmax
 };
@@ -101,7 +102,7 @@ struct FwdShape {
 constexpr int kMaxKeyBlocks = 4096;
 
 template <int KS, int VS>
-struct alignas(8) FwdBarriers {
+struct alignas(16) FwdBarriers {
   uint64_t q_full;
   uint64_t k_full[KS], k_empty[KS];
   uint64_t v_full[VS], v_empty[VS];
@@ -377,7 +378,7 @@ struct SoftmaxRow {
 // earlier block was abandoned: 'failed'), which every softmax thread learns
 // after the same barrier, else 0. An abandoned step still takes part in both
 // barriers, so the barrier accounting of the softmax and waiter warps agrees.
-template <int D, int BQ, int BK, bool CAUSAL, bool WRITE_MASK, typename Bars>
+template <int D, int BQ, int BK, bool CAUSAL, bool WRITE_MASK, bool GAP, typename Bars>
 __device__ __forceinline__ int softmax_block(const FwdParams& p, Bars* bars, uint32_t tmem, const FwdUnit& w,
                                              int s, int j, float tau, SoftmaxRow<BK>& st, bool failed) {
   using S = FwdShape<D, BQ, BK>;
@@ -444,8 +445,8 @@ __device__ __forceinline__ int softmax_block(const FwdParams& p, Bars* bars, uin
   const float run_max = s ? st.M[1] : st.M[0];
   const bool above =
       ok && qrow < p.N &&
-      (p.gate_gap ? (pmax > -INFINITY && (run_max == -INFINITY || pmax * p.scale_log2 >= run_max - tau))
-                  : (pmax * p.scale >= tau));
+      (GAP ? (pmax > -INFINITY && (run_max == -INFINITY || pmax * p.scale_log2 >= run_max - tau))
+           : (pmax * p.scale >= tau));
   bool any_above[S::NSUB];
   any_above[0] = named_barrier_or(kGateBar, 32 * kSoftmaxWarps, above && (S::NSUB == 1 || sub == 0));
   if constexpr (S::NSUB == 2) any_above[1] = named_barrier_or(kGateBar, 32 * kSoftmaxWarps, above && sub == 1);
@@ -494,7 +495,9 @@ __device__ __forceinline__ int softmax_block(const FwdParams& p, Bars* bars, uin
   float alpha = 1.f;
   if (my_keep) {
     const float mx = rmax * p.scale_log2;
-    if (s) st.M[1] = fmaxf(st.M[1], mx); else st.M[0] = fmaxf(st.M[0], mx);
+    if (GAP) {
+      if (s) st.M[1] = fmaxf(st.M[1], mx); else st.M[0] = fmaxf(st.M[0], mx);
+    }
     if (mx > m + kRescaleThreshold) {      // also taken on the first finite maximum
       if (m != -INFINITY) {
         alpha = ex2_approx(m - mx);
@@ -611,7 +614,7 @@ __device__ __forceinline__ void softmax_epilogue(const FwdParams& p, Bars* bars,
     p.lse[(size_t)(w.b * p.Hq + hq) * p.N + qrow] = (m + __log2f(l_row)) * 0.69314718055994531f;
 }
 
-template <int D, int BQ, int BK, bool CAUSAL, bool WRITE_MASK, typename Bars>
+template <int D, int BQ, int BK, bool CAUSAL, bool WRITE_MASK, bool GAP, typename Bars>
 __device__ __forceinline__ void softmax_role(const FwdParams& p, Bars* bars, uint32_t tmem, const FwdUnit& w) {
   SoftmaxRow<BK> st;
   bool aborted = false;
@@ -622,7 +625,7 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, Bars* bars, uin
     const int hq = w.hq[s];
     const int tile = w.q0[s] / BQ + sub;
     const float t = p.tau_tiles > 0 ? p.tau[hq * p.tau_tiles + min(tile, p.tau_tiles - 1)] : p.tau[hq];
-    return p.gate_gap ? t * 1.4426950408889634f : t;   // gamma in the exp2 domain of the running maximum
+    return GAP ? t * 1.4426950408889634f : t;   // gamma in the exp2 domain of the running maximum
   };
   const float tau0 = tile_tau(0), tau1 = tile_tau(1);
   const int nblk = max(w.nblk[0], w.nblk[1]);
@@ -632,7 +635,7 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, Bars* bars, uin
 #pragma unroll 1
     for (int s = 0; s < 2; ++s) {
       if (j >= (s ? w.nblk[1] : w.nblk[0])) continue;
-      if (softmax_block<D, BQ, BK, CAUSAL, WRITE_MASK>(p, bars, tmem, w, s, j, s ? tau1 : tau0, st, aborted) == 2)
+      if (softmax_block<D, BQ, BK, CAUSAL, WRITE_MASK, GAP>(p, bars, tmem, w, s, j, s ? tau1 : tau0, st, aborted) == 2)
         aborted = true;
     }
   }
@@ -645,7 +648,7 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, Bars* bars, uin
 
 // ---------------------------------------------------------------------------- kernel
 
-template <int D, int BQ, int BK, bool CAUSAL, bool WRITE_MASK>
+template <int D, int BQ, int BK, bool CAUSAL, bool WRITE_MASK, bool GAP>
 __global__ void __launch_bounds__(kThreads, 1)
     bsfa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -691,7 +694,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < kSoftmaxWarps) {
     regs_increase<kSoftmaxRegs>();
-    softmax_role<D, BQ, BK, CAUSAL, WRITE_MASK>(p, bars, tmem, w);
+    softmax_role<D, BQ, BK, CAUSAL, WRITE_MASK, GAP>(p, bars, tmem, w);
   } else {
     regs_decrease<kProducerRegs>();
     if (lane == 0) {

@@ -1,5 +1,5 @@
 // Kernel instantiation and launch for one head dimension (used by the per-D
-// translation units so the 32 kernel variants compile in parallel).
+// translation units so the 64 kernel variants compile in parallel).
 #pragma once
 
 #include <cuda_runtime.h>
@@ -8,11 +8,11 @@
 
 namespace bsfa {
 
-template <int D, int BQ, int BK, bool CAUSAL, bool MASK>
+template <int D, int BQ, int BK, bool CAUSAL, bool MASK, bool GAP>
 cudaError_t launch_variant(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
                            int grid, cudaStream_t stream) {
   using S = FwdShape<D, BQ, BK>;
-  auto kern = bsfa_fwd_kernel<D, BQ, BK, CAUSAL, MASK>;
+  auto kern = bsfa_fwd_kernel<D, BQ, BK, CAUSAL, MASK, GAP>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   kern<<<grid, kThreads, S::SMEM_BYTES, stream>>>(tq, tk, tv, p);
@@ -24,11 +24,18 @@ cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
                        int Bq, int Bk, bool causal, bool mask, int grid, cudaStream_t s) {
 #define BSFA_CASE(BQ, BK)                                                                          \
   if (Bq == BQ && Bk == BK) {                                                                      \
+    if (p.gate_gap) {                                                                              \
+      if (causal)                                                                                  \
+        return mask ? launch_variant<D, BQ, BK, true, true, true>(tq, tk, tv, p, grid, s)          \
+                    : launch_variant<D, BQ, BK, true, false, true>(tq, tk, tv, p, grid, s);        \
+      return mask ? launch_variant<D, BQ, BK, false, true, true>(tq, tk, tv, p, grid, s)           \
+                  : launch_variant<D, BQ, BK, false, false, true>(tq, tk, tv, p, grid, s);         \
+    }                                                                                              \
     if (causal)                                                                                    \
-      return mask ? launch_variant<D, BQ, BK, true, true>(tq, tk, tv, p, grid, s)                  \
-                  : launch_variant<D, BQ, BK, true, false>(tq, tk, tv, p, grid, s);                \
-    return mask ? launch_variant<D, BQ, BK, false, true>(tq, tk, tv, p, grid, s)                   \
-                : launch_variant<D, BQ, BK, false, false>(tq, tk, tv, p, grid, s);                 \
+      return mask ? launch_variant<D, BQ, BK, true, true, false>(tq, tk, tv, p, grid, s)           \
+                  : launch_variant<D, BQ, BK, true, false, false>(tq, tk, tv, p, grid, s);         \
+    return mask ? launch_variant<D, BQ, BK, false, true, false>(tq, tk, tv, p, grid, s)            \
+                : launch_variant<D, BQ, BK, false, false, false>(tq, tk, tv, p, grid, s);          \
   }
   BSFA_CASE(64, 64)
   BSFA_CASE(64, 128)
