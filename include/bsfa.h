@@ -118,6 +118,36 @@ bsfa_status bsfa_forward_gap(const void* q, const void* k, const void* v, const 
                              void* stream);
 
 /*
+ * bsfa_forward_varlen - bsfa_forward over a packed batch of sequences of
+ * different lengths (mixed-length prefill). Sequence e holds rows
+ * [cu_seqlens[e], cu_seqlens[e+1]) of the packed tensors; each sequence is its
+ * own attention problem, tiled from its own first row (App. B.2 tiling applied
+ * per sequence).
+ *
+ *   q          bf16 [total, Hq,  D], contiguous, device memory, 16-byte aligned (read)
+ *   k, v       bf16 [total, Hkv, D], contiguous, device memory, 16-byte aligned (read)
+ *   cu_seqlens int32 [nseq + 1], device memory: cu_seqlens[0] = 0, non-decreasing,
+ *              cu_seqlens[nseq] <= total. Offsets outside [0, total] are clamped and a
+ *              sequence longer than max_seqlen is cut to max_seqlen (its rows past that
+ *              are not written), so bad offsets cannot make the kernel leave the buffers.
+ *   nseq       number of sequences, >= 1
+ *   max_seqlen length of the longest sequence (it sizes the grid), >= 1, with
+ *              ceil(max_seqlen / Bk) <= 4096
+ *   tau        fp32 [Hq], device memory (one threshold per head)
+ *   out        bf16 [total, Hq, D], device memory (written for the rows of every sequence)
+ *   lse        fp32 [Hq, total], device memory, or NULL
+ *   block_mask uint8 [nseq, Hq, ceil(max_seqlen/Bq), ceil(max_seqlen/Bk)], device
+ *              memory, or NULL; entries past a sequence's own tiles stay 3
+ *   total      total rows of the packed tensors
+ *
+ * Hq, Hkv, D, Bq, Bk, causal and stream, the supported set and the error
+ * behaviour are those of bsfa_forward.
+ */
+bsfa_status bsfa_forward_varlen(const void* q, const void* k, const void* v, const int* cu_seqlens, int nseq,
+                                int max_seqlen, const float* tau, void* out, float* lse, uint8_t* block_mask,
+                                int total, int Hq, int Hkv, int D, int Bq, int Bk, int causal, void* stream);
+
+/*
  * bsfa_validate - the shape checks of bsfa_forward, host only (no CUDA call).
  * Returns BSFA_OK, BSFA_ERR_INVALID_ARG or BSFA_ERR_UNSUPPORTED.
  */

@@ -309,3 +309,24 @@ def block_maxima(q_bits, k_bits, Bq: int, Bk: int, causal: bool, tiles=None) -> 
         t = forward_tile(q_bits, k_bits, None, tau_inf, b, hq, i, Bq, Bk, causal, with_output=False)
         res[(b, hq, i)] = (t["codes"], t["smax"])
     return res
+
+
+def forward_varlen(q_bits, k_bits, v_bits, cu_seqlens, tau, Bq: int, Bk: int, causal: bool) -> dict:
+    """A packed batch of sequences of different lengths: each sequence
+    [cu[e], cu[e+1]) of q [total, Hq, D] and k, v [total, Hkv, D] is its own
+    forward (App. B.2 tiling starts at its first row). Returns out [total, Hq, D],
+    lse [Hq, total] and, per sequence, its codes [Hq, M_Q, M_KV]."""
+    total, Hq, D = q_bits.shape
+    out = np.zeros((total, Hq, D))
+    lse = np.zeros((Hq, total))
+    codes = []
+    for e in range(len(cu_seqlens) - 1):
+        r0, r1 = int(cu_seqlens[e]), int(cu_seqlens[e + 1])
+        if r1 <= r0:
+            codes.append(None)
+            continue
+        r = forward(q_bits[None, r0:r1], k_bits[None, r0:r1], v_bits[None, r0:r1], tau, Bq, Bk, causal)
+        out[r0:r1] = r["out"][0]
+        lse[:, r0:r1] = r["lse"][0]
+        codes.append(r["codes"][0])
+    return {"out": out, "lse": lse, "codes": codes}

@@ -85,3 +85,15 @@ def test_tau_table_entry_rejects_bad_arguments_without_touching_cuda(lib):
         assert "tau_tiles" in bsfa.bsfa_last_error()
     assert bsfa.bsfa_forward_tau_table(16, 16, 16, None, 4, 16, None, None, *shape, None) == bsfa.BSFA_ERR_INVALID_ARG
     assert bsfa.bsfa_forward_tau_table(16, 16, 16, 18, 4, 16, None, None, *shape, None) == bsfa.BSFA_ERR_INVALID_ARG
+
+
+def test_varlen_entry_rejects_bad_arguments_without_touching_cuda(lib):
+    args = dict(total=1000, Hq=4, Hkv=2, D=128, Bq=128, Bk=128, causal=1)
+    call = lambda cu, nseq, max_len, D=128: bsfa.bsfa_forward_varlen(16, 16, 16, cu, nseq, max_len, 16, 16, None, None,
+                                                                      1000, 4, 2, D, 128, 128, 1, None)
+    assert call(None, 2, 500) == bsfa.BSFA_ERR_INVALID_ARG          # no offsets
+    assert call(16, 0, 500) == bsfa.BSFA_ERR_INVALID_ARG            # no sequences
+    assert call(16, 2, 0) == bsfa.BSFA_ERR_INVALID_ARG              # no length
+    assert call(18, 2, 500) == bsfa.BSFA_ERR_INVALID_ARG            # misaligned offsets
+    assert call(16, 2, 4097 * 128) == bsfa.BSFA_ERR_UNSUPPORTED     # too many key blocks
+    assert call(16, 2, 500, D=96) == bsfa.BSFA_ERR_UNSUPPORTED      # head dimension

@@ -6,7 +6,8 @@ fallback: if the library is missing or the device is not sm_100, calls fail
 loudly.
 
 The functions named like the C entry points (``bsfa_forward``,
-``bsfa_forward_tau_table``, ``bsfa_forward_gap``, ``bsfa_validate``, ``bsfa_get_status``,
+``bsfa_forward_tau_table``, ``bsfa_forward_gap``, ``bsfa_forward_varlen``, ``bsfa_validate``,
+``bsfa_get_status``,
 ``bsfa_selftest_lost_arrival``, ``bsfa_status_string``, ``bsfa_last_error``)
 take the same arguments; pointer arguments accept an int
 address, None, or a torch tensor (its ``data_ptr()``). ``forward`` and
@@ -26,7 +27,8 @@ BSFA_ERR_UNSUPPORTED = 2
 BSFA_ERR_CUDA = 3
 BSFA_ERR_DEVICE_TIMEOUT = 4
 
-EXPORTED = ("bsfa_forward", "bsfa_forward_tau_table", "bsfa_forward_gap", "bsfa_validate", "bsfa_get_status",
+EXPORTED = ("bsfa_forward", "bsfa_forward_tau_table", "bsfa_forward_gap", "bsfa_forward_varlen", "bsfa_validate",
+            "bsfa_get_status",
             "bsfa_selftest_lost_arrival", "bsfa_status_string", "bsfa_last_error")
 
 _lib = None
@@ -53,6 +55,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.bsfa_forward_tau_table.restype = i
     lib.bsfa_forward_gap.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, vp]
     lib.bsfa_forward_gap.restype = i
+    lib.bsfa_forward_varlen.argtypes = [vp, vp, vp, vp, i, i, vp, vp, vp, vp, i, i, i, i, i, i, i, vp]
+    lib.bsfa_forward_varlen.restype = i
     lib.bsfa_validate.argtypes = [i] * 8
     lib.bsfa_validate.restype = i
     lib.bsfa_get_status.argtypes = [vp]
@@ -100,6 +104,13 @@ def bsfa_forward_tau_table(q, k, v, tau_table, tau_tiles, out, lse, block_mask, 
 def bsfa_forward_gap(q, k, v, gamma, out, lse, block_mask, B, Hq, Hkv, N, D, Bq, Bk, causal, stream) -> int:
     return load().bsfa_forward_gap(_ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(out), _ptr(lse), _ptr(block_mask),
                                    B, Hq, Hkv, N, D, Bq, Bk, int(bool(causal)), _stream(stream))
+
+
+def bsfa_forward_varlen(q, k, v, cu_seqlens, nseq, max_seqlen, tau, out, lse, block_mask, total, Hq, Hkv, D, Bq, Bk,
+                        causal, stream) -> int:
+    return load().bsfa_forward_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), int(nseq), int(max_seqlen),
+                                      _ptr(tau), _ptr(out), _ptr(lse), _ptr(block_mask), total, Hq, Hkv, D, Bq, Bk,
+                                      int(bool(causal)), _stream(stream))
 
 
 def bsfa_validate(B, Hq, Hkv, N, D, Bq, Bk, causal) -> int:
@@ -170,6 +181,32 @@ def forward(q, k, v, tau, *, Bq: int, Bk: int, causal: bool, want_lse: bool = Tr
         _check(bsfa_forward_tau_table(q, k, v, tau, tau.shape[1], out, lse_arg, mask_arg, B, Hq, Hkv, N, D, Bq, Bk,
                                       causal, stream))
     return out, (lse if want_lse else None), (block_mask if want_mask else None)
+
+
+def forward_varlen(q, k, v, cu_seqlens, max_seqlen: int, tau, *, Bq: int, Bk: int, causal: bool,
+                   want_lse: bool = True, want_mask: bool = False, stream=None):
+    """Packed mixed-length batch on device tensors. q: bf16 [total, Hq, D]; k, v: bf16
+    [total, Hkv, D]; cu_seqlens: int32 [nseq + 1] CUDA tensor; tau: fp32 [Hq].
+    Returns (out [total, Hq, D], lse [Hq, total] or None, block_mask or None)."""
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or t.dim() != 3:
+            raise ValueError(f"{name} must be a contiguous 3-D bf16 CUDA tensor")
+    if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_cuda or cu_seqlens.dim() != 1:
+        raise ValueError("cu_seqlens must be a 1-D int32 CUDA tensor")
+    total, Hq, D = q.shape
+    Hkv = k.shape[1]
+    nseq = cu_seqlens.numel() - 1
+    out = torch.empty_like(q)
+    lse = torch.empty((Hq, total), dtype=torch.float32, device=q.device) if want_lse else None
+    mask = None
+    if want_mask:
+        mask = torch.empty((nseq, Hq, -(-max_seqlen // Bq), -(-max_seqlen // Bk)), dtype=torch.uint8, device=q.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    _check(bsfa_forward_varlen(q, k, v, cu_seqlens, nseq, max_seqlen, tau, out, lse, mask, total, Hq, Hkv, D, Bq, Bk,
+                               causal, stream))
+    return out, lse, mask
 
 
 def forward_host(q, k, v, tau, *, Bq: int, Bk: int, causal: bool, device=None, stream=None, bufs=None,

@@ -128,12 +128,25 @@ bsfa_status bsfa_validate(int B, int Hq, int Hkv, int N, int D, int Bq, int Bk, 
 namespace {
 
 // Every forward entry point: tau_tiles == 0 selects one value per head; gate_gap
-// selects the gap gate, tau then holding gamma.
+// selects the gap gate, tau then holding gamma. With cu_seqlens the input is B
+// packed sequences of at most max_seqlen rows in N = total rows.
 bsfa_status forward_impl(const void* q, const void* k, const void* v, const float* tau, int tau_tiles, int gate_gap,
                          void* out, float* lse, uint8_t* block_mask, int B, int Hq, int Hkv, int N, int D, int Bq,
-                         int Bk, int causal, void* stream) {
-  bsfa_status st = bsfa_validate(B, Hq, Hkv, N, D, Bq, Bk, causal);
+                         int Bk, int causal, void* stream, const int* cu_seqlens = nullptr, int max_seqlen = 0) {
+  bsfa_status st = cu_seqlens ? bsfa_validate(1, Hq, Hkv, N, D, Bq, Bk, causal)
+                              : bsfa_validate(B, Hq, Hkv, N, D, Bq, Bk, causal);
   if (st != BSFA_OK) return st;
+  if (cu_seqlens) {
+    if (B <= 0 || max_seqlen <= 0) return fail(BSFA_ERR_INVALID_ARG, "nseq=%d and max_seqlen=%d must be positive", B, max_seqlen);
+    if (!aligned(cu_seqlens, 4)) return fail(BSFA_ERR_INVALID_ARG, "cu_seqlens must be 4-byte aligned");
+    const long long key_blocks = ((long long)max_seqlen + Bk - 1) / Bk;
+    if (key_blocks > bsfa::kMaxKeyBlocks)
+      return fail(BSFA_ERR_UNSUPPORTED, "ceil(max_seqlen/Bk)=%lld exceeds %d key blocks", key_blocks, bsfa::kMaxKeyBlocks);
+    if ((long long)B * Hq * (((long long)max_seqlen + 127) / 128) > 0x7fffffffLL)
+      return fail(BSFA_ERR_UNSUPPORTED, "nseq * Hq * ceil(max_seqlen/128) exceeds the grid");
+  } else {
+    max_seqlen = N;
+  }
   if (tau_tiles < 0) return fail(BSFA_ERR_INVALID_ARG, "tau_tiles=%d is negative", tau_tiles);
   if (!q || !k || !v || !tau || !out) return fail(BSFA_ERR_INVALID_ARG, "q, k, v, tau and out must be non-null");
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16))
@@ -149,20 +162,25 @@ bsfa_status forward_impl(const void* q, const void* k, const void* v, const floa
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (block_mask) {
-    const size_t n = (size_t)B * Hq * (size_t)((N + Bq - 1) / Bq) * (size_t)((N + Bk - 1) / Bk);
+    const size_t n = (size_t)B * Hq * (size_t)((max_seqlen + Bq - 1) / Bq) * (size_t)((max_seqlen + Bk - 1) / Bk);
     e = cudaMemsetAsync(block_mask, 3, n, s);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(block_mask)");
   }
 
   CUtensorMap tq, tk, tv;
-  if (!encode_bnhd(&tq, q, B, N, Hq, D, 128) || !encode_bnhd(&tk, k, B, N, Hkv, D, Bk) ||
-      !encode_bnhd(&tv, v, B, N, Hkv, D, Bk))
+  const int map_b = cu_seqlens ? 1 : B;     // packed sequences are one batch entry of N rows
+  if (!encode_bnhd(&tq, q, map_b, N, Hq, D, 128) || !encode_bnhd(&tk, k, map_b, N, Hkv, D, Bk) ||
+      !encode_bnhd(&tv, v, map_b, N, Hkv, D, Bk))
     return fail(BSFA_ERR_CUDA, "cuTensorMapEncodeTiled failed");
 
   bsfa::FwdParams p;
   p.tau = tau;
   p.tau_tiles = tau_tiles;
   p.gate_gap = gate_gap;
+  p.cu_seqlens = cu_seqlens;
+  p.max_seqlen = max_seqlen;
+  p.mask_mq = (max_seqlen + Bq - 1) / Bq;
+  p.mask_mkv = (max_seqlen + Bk - 1) / Bk;
   p.out = static_cast<uint16_t*>(out);
   p.lse = lse;
   p.mask = block_mask;
@@ -177,7 +195,7 @@ bsfa_status forward_impl(const void* q, const void* k, const void* v, const floa
   p.pair_heads = (p.group % 2 == 0) ? 1 : 0;
   p.scale = (float)(1.0 / std::sqrt((double)D));
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
-  const int tiles = (N + 127) / 128;
+  const int tiles = (max_seqlen + 127) / 128;
   const int grid = p.pair_heads ? B * (Hq / 2) * tiles : B * Hq * ((tiles + 1) / 2);
   e = (D == 64) ? bsfa::launch_fwd_d64(tq, tk, tv, p, Bq, Bk, causal != 0, block_mask != nullptr, grid, s)
                 : bsfa::launch_fwd_d128(tq, tk, tv, p, Bq, Bk, causal != 0, block_mask != nullptr, grid, s);
@@ -207,6 +225,14 @@ bsfa_status bsfa_forward_gap(const void* q, const void* k, const void* v, const 
                              uint8_t* block_mask, int B, int Hq, int Hkv, int N, int D, int Bq, int Bk, int causal,
                              void* stream) {
   return forward_impl(q, k, v, gamma, 0, 1, out, lse, block_mask, B, Hq, Hkv, N, D, Bq, Bk, causal, stream);
+}
+
+bsfa_status bsfa_forward_varlen(const void* q, const void* k, const void* v, const int* cu_seqlens, int nseq,
+                                int max_seqlen, const float* tau, void* out, float* lse, uint8_t* block_mask,
+                                int total, int Hq, int Hkv, int D, int Bq, int Bk, int causal, void* stream) {
+  if (!cu_seqlens) return fail(BSFA_ERR_INVALID_ARG, "cu_seqlens must be non-null");
+  return forward_impl(q, k, v, tau, 0, 0, out, lse, block_mask, nseq, Hq, Hkv, total, D, Bq, Bk, causal, stream,
+                      cu_seqlens, max_seqlen);
 }
 
 bsfa_status bsfa_get_status(void* stream) {

@@ -44,6 +44,12 @@ struct FwdParams {
   uint8_t* mask;      // [B, Hq, N/Bq, N/Bk] or null
   int* status;        // device status word
   int B, Hq, Hkv, N;  // N need not be a multiple of the tile sizes: rows and keys >= N are masked
+  // Packed variable-length batch (the kernel's VARLEN variants; null otherwise):
+  // sequence e holds rows [cu_seqlens[e], cu_seqlens[e+1]) of the N = total rows,
+  // and B is the sequence count.
+  const int* cu_seqlens;
+  int max_seqlen;     // longest sequence (N for [B, N] inputs): sizes the grid
+  int mask_mq, mask_mkv;   // query tiles and key blocks per sequence in the block mask
   int group;          // Hq / Hkv
   int pair_heads;     // 1: slots are query heads 2p and 2p+1 on the same rows
   int gate_gap;       // 0: the BSFA gate (block maximum against tau); 1: the gap gate, tau holding gamma
@@ -117,11 +123,18 @@ struct alignas(16) FwdBarriers {
 
 struct FwdUnit {
   int b, kvh;
-  int hq[2], q0[2], nblk[2];
+  int hq[2], q0[2], nblk[2];   // q0: first row of the slot within its sequence
 };
 
-__device__ __forceinline__ FwdUnit decode_unit(const FwdParams& p, int u, bool causal, int bk) {
-  const int tiles = (p.N + 127) / 128;
+// Where a unit's sequence lies among packed sequences (VARLEN variants only).
+struct SeqSpan {
+  int row0, len;               // the sequence's first row in the N dimension, and its length
+  int seq;                     // the sequence's index
+};
+
+template <bool VARLEN>
+__device__ __forceinline__ FwdUnit decode_unit(const FwdParams& p, int u, bool causal, int bk, SeqSpan& sp) {
+  const int tiles = ((VARLEN ? p.max_seqlen : p.N) + 127) / 128;
   FwdUnit w;
   if (p.pair_heads) {
     // Consecutive units: the head pairs of one row block, a KV group's pairs adjacent.
@@ -144,11 +157,29 @@ __device__ __forceinline__ FwdUnit decode_unit(const FwdParams& p, int u, bool c
     w.q0[1] = w.q0[0] + 128;
   }
   w.kvh = w.hq[0] / p.group;
+  int len = p.N;
+  if (VARLEN) {   // packed sequences: one batch entry of N = total rows
+    // Offsets are clamped to [0, N] and lengths to max_seqlen, so no access can
+    // leave the caller's buffers whatever the offsets hold.
+    sp.seq = w.b;
+    sp.row0 = min(max(p.cu_seqlens[w.b], 0), p.N);
+    sp.len = len = min(min(max(p.cu_seqlens[w.b + 1], sp.row0), p.N) - sp.row0, p.max_seqlen);
+    w.b = 0;
+  }
 #pragma unroll
   for (int s = 0; s < 2; ++s)
-    w.nblk[s] = (w.q0[s] >= p.N) ? 0 : (causal ? min((w.q0[s] + 128) / bk, (p.N + bk - 1) / bk) : (p.N + bk - 1) / bk);
+    w.nblk[s] = (w.q0[s] >= len) ? 0 : (causal ? min((w.q0[s] + 128) / bk, (len + bk - 1) / bk) : (len + bk - 1) / bk);
   return w;
 }
+
+// The unit's sequence length, first row and index. For [B, N] inputs these are
+// compile-time forms of N, 0 and b, and the span is never read.
+template <bool VARLEN>
+__device__ __forceinline__ int unit_len(const SeqSpan& sp, const FwdParams& p) { return VARLEN ? sp.len : p.N; }
+template <bool VARLEN>
+__device__ __forceinline__ int unit_row0(const SeqSpan& sp) { return VARLEN ? sp.row0 : 0; }
+template <bool VARLEN>
+__device__ __forceinline__ int unit_seq(const FwdUnit& w, const SeqSpan& sp) { return VARLEN ? sp.seq : w.b; }
 
 // Bounded wait used when draining in-flight copies/MMAs on the way out: it does
 // not give up early on the abort flag, only on the time limit.
@@ -159,9 +190,9 @@ __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
 
 // ---------------------------------------------------------------------------- K/Q producer (warp 8, one thread)
 
-template <int D, int BQ, int BK, typename Bars>
+template <int D, int BQ, int BK, bool VARLEN, typename Bars>
 __device__ __forceinline__ void kq_producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k, uint8_t* smem,
-                                            Bars* bars, const FwdUnit& w) {
+                                            Bars* bars, const FwdUnit& w, const SeqSpan& sp) {
   using S = FwdShape<D, BQ, BK>;
   volatile int* abort_flag = &bars->abort;
   prefetch_tensormap(tm_q);
@@ -174,7 +205,7 @@ __device__ __forceinline__ void kq_producer(const CUtensorMap* tm_q, const CUten
 #pragma unroll
     for (int c = 0; c < S::DCH; ++c)
       tma_load_4d(smem + S::OFF_Q + s * S::Q_BYTES + c * (S::ROWS * 128), tm_q, &bars->q_full, c * 64, w.hq[s],
-                  w.q0[s], w.b);
+                  unit_row0<VARLEN>(sp) + w.q0[s], w.b);
   }
   const int nblk = max(w.nblk[0], w.nblk[1]);
   int issued = 0;
@@ -185,7 +216,7 @@ __device__ __forceinline__ void kq_producer(const CUtensorMap* tm_q, const CUten
 #pragma unroll
     for (int c = 0; c < S::DCH; ++c)
       tma_load_4d(smem + S::OFF_K + slot * S::KV_BYTES + c * (BK * 128), tm_k, &bars->k_full[slot], c * 64, w.kvh,
-                  t * BK, w.b);
+                  unit_row0<VARLEN>(sp) + t * BK, w.b);
     issued = t + 1;
   }
   // Copies still in flight must land before the CTA exits.
@@ -216,8 +247,9 @@ __device__ __forceinline__ bool wait_decided(Bars* bars, int s, int j) {
 
 // ---------------------------------------------------------------------------- V producer (one thread)
 
-template <int D, int BQ, int BK, typename Bars>
-__device__ __forceinline__ void v_producer(const CUtensorMap* tm_v, uint8_t* smem, Bars* bars, const FwdUnit& w) {
+template <int D, int BQ, int BK, bool VARLEN, typename Bars>
+__device__ __forceinline__ void v_producer(const CUtensorMap* tm_v, uint8_t* smem, Bars* bars, const FwdUnit& w,
+                                           const SeqSpan& sp) {
   using S = FwdShape<D, BQ, BK>;
   volatile int* abort_flag = &bars->abort;
   prefetch_tensormap(tm_v);
@@ -238,7 +270,7 @@ __device__ __forceinline__ void v_producer(const CUtensorMap* tm_v, uint8_t* sme
 #pragma unroll
       for (int c = 0; c < S::DCH; ++c)
         tma_load_4d(smem + S::OFF_V + slot * S::KV_BYTES + c * (BK * 128), tm_v, &bars->v_full[slot], c * 64, w.kvh,
-                    j * BK, w.b);
+                    unit_row0<VARLEN>(sp) + j * BK, w.b);
       loaded = true;
     }
     if (loaded) ++v_count;
@@ -378,9 +410,10 @@ struct SoftmaxRow {
 // earlier block was abandoned: 'failed'), which every softmax thread learns
 // after the same barrier, else 0. An abandoned step still takes part in both
 // barriers, so the barrier accounting of the softmax and waiter warps agrees.
-template <int D, int BQ, int BK, bool CAUSAL, bool WRITE_MASK, bool GAP, typename Bars>
+template <int D, int BQ, int BK, bool CAUSAL, bool WRITE_MASK, bool GAP, bool VARLEN, typename Bars>
 __device__ __forceinline__ int softmax_block(const FwdParams& p, Bars* bars, uint32_t tmem, const FwdUnit& w,
-                                             int s, int j, float tau, SoftmaxRow<BK>& st, bool failed) {
+                                             const SeqSpan& sp, int s, int j, float tau, SoftmaxRow<BK>& st,
+                                             bool failed) {
   using S = FwdShape<D, BQ, BK>;
   constexpr int QC = BK / kRowSplit;         // key columns per thread
   constexpr int QD = D / kRowSplit;          // output columns per thread
@@ -419,7 +452,7 @@ __device__ __forceinline__ int softmax_block(const FwdParams& p, Bars* bars, uin
     // causal padding row (qrow >= N) also sees the zero-filled keys up to qrow;
     // it is left out of the gate and never written, and V is zero there.
     const int k0 = j * BK + c4 * QC;
-    const int klim = CAUSAL ? qrow : p.N - 1;
+    const int klim = CAUSAL ? qrow : unit_len<VARLEN>(sp, p) - 1;
     if (k0 + QC - 1 > klim) {                    // this thread's columns reach past it
 #pragma unroll
       for (int c = 0; c < QC; ++c)
@@ -444,7 +477,7 @@ __device__ __forceinline__ int softmax_block(const FwdParams& p, Bars* bars, uin
   // maximum minus gamma.
   const float run_max = s ? st.M[1] : st.M[0];
   const bool above =
-      ok && qrow < p.N &&
+      ok && qrow < unit_len<VARLEN>(sp, p) &&
       (GAP ? (pmax > -INFINITY && (run_max == -INFINITY || pmax * p.scale_log2 >= run_max - tau))
            : (pmax * p.scale >= tau));
   bool any_above[S::NSUB];
@@ -463,18 +496,19 @@ __device__ __forceinline__ int softmax_block(const FwdParams& p, Bars* bars, uin
     // holding a row's own key is forced even in a last tile of one row.
     const int lo = q0 + t * BQ;
     const int k_lo = j * BK;
-    const bool visible = lo < p.N && (!CAUSAL || k_lo <= min(lo + BQ - 1, p.N - 1));
+    const int len = unit_len<VARLEN>(sp, p);
+    const bool visible = lo < len && (!CAUSAL || k_lo <= min(lo + BQ - 1, len - 1));
     const bool diag = visible && (CAUSAL ? k_lo + BK - 1 > lo : (k_lo < lo + BQ && k_lo + BK > lo));
     code[t] = !visible ? 3 : diag ? 2 : (any_above[t] ? 1 : 0);
     keep_any |= (code[t] == 1 || code[t] == 2);
   }
   if (warp == 0 && lane == 0) {
     if (WRITE_MASK) {
-      const int mq = (p.N + BQ - 1) / BQ, mkv = (p.N + BK - 1) / BK;
+      const int mq = p.mask_mq, mkv = p.mask_mkv;
 #pragma unroll
       for (int t = 0; t < S::NSUB; ++t)
         if (code[t] != 3)
-          p.mask[((size_t)(w.b * p.Hq + hq) * mq + (q0 / BQ + t)) * mkv + j] = (uint8_t)code[t];
+          p.mask[((size_t)(unit_seq<VARLEN>(w, sp) * p.Hq + hq) * mq + (q0 / BQ + t)) * mkv + j] = (uint8_t)code[t];
     }
     // Publish the decision (one byte, no fence) so the V tile, if kept, is fetched
     // right away; the MMA warp reads it after p_full, whose arrival orders it.
@@ -559,9 +593,9 @@ __device__ __forceinline__ int softmax_block(const FwdParams& p, Bars* bars, uin
 // Epilogue of one slot: the two threads of each row combine their normalisers
 // through shared memory, then each writes its D/2 output columns; lse is the
 // natural-log logsumexp over the kept set.
-template <int D, int BQ, int BK, typename Bars>
+template <int D, int BQ, int BK, bool VARLEN, typename Bars>
 __device__ __forceinline__ void softmax_epilogue(const FwdParams& p, Bars* bars, uint32_t tmem, const FwdUnit& w,
-                                                 int s, SoftmaxRow<BK>& st, bool failed) {
+                                                 const SeqSpan& sp, int s, SoftmaxRow<BK>& st, bool failed) {
   using S = FwdShape<D, BQ, BK>;
   constexpr int QD = D / kRowSplit;
   volatile int* abort_flag = &bars->abort;
@@ -591,9 +625,9 @@ __device__ __forceinline__ void softmax_epilogue(const FwdParams& p, Bars* bars,
   const uint32_t o_tmem = tmem + S::TMEM_O0 + s * D + c4 * QD + ((uint32_t)(q * 32) << 16);
   // Padding rows of a last tile (qrow >= N) take part in the warp's TMEM loads
   // (warp-collective) but store nothing.
-  const bool row_ok = qrow < p.N;
+  const bool row_ok = qrow < unit_len<VARLEN>(sp, p);
   const float inv_l = 1.f / l_row;     // > 0: every row keeps its diagonal block, which holds its own key
-  uint16_t* orow = p.out + ((size_t)(w.b * p.N + qrow) * p.Hq + hq) * D + c4 * QD;
+  uint16_t* orow = p.out + ((size_t)(w.b * p.N + unit_row0<VARLEN>(sp) + qrow) * p.Hq + hq) * D + c4 * QD;
 #pragma unroll
   for (int c = 0; c < QD / 32 + (QD < 32); ++c) {
     constexpr int W = QD < 32 ? QD : 32;
@@ -611,11 +645,12 @@ __device__ __forceinline__ void softmax_epilogue(const FwdParams& p, Bars* bars,
     }
   }
   if (row_ok && c4 == 0 && p.lse != nullptr)
-    p.lse[(size_t)(w.b * p.Hq + hq) * p.N + qrow] = (m + __log2f(l_row)) * 0.69314718055994531f;
+    p.lse[(size_t)(w.b * p.Hq + hq) * p.N + unit_row0<VARLEN>(sp) + qrow] = (m + __log2f(l_row)) * 0.69314718055994531f;
 }
 
-template <int D, int BQ, int BK, bool CAUSAL, bool WRITE_MASK, bool GAP, typename Bars>
-__device__ __forceinline__ void softmax_role(const FwdParams& p, Bars* bars, uint32_t tmem, const FwdUnit& w) {
+template <int D, int BQ, int BK, bool CAUSAL, bool WRITE_MASK, bool GAP, bool VARLEN, typename Bars>
+__device__ __forceinline__ void softmax_role(const FwdParams& p, Bars* bars, uint32_t tmem, const FwdUnit& w,
+                                             const SeqSpan& sp) {
   SoftmaxRow<BK> st;
   bool aborted = false;
   // This thread's threshold in each slot: its query tile's column of the table
@@ -635,20 +670,21 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, Bars* bars, uin
 #pragma unroll 1
     for (int s = 0; s < 2; ++s) {
       if (j >= (s ? w.nblk[1] : w.nblk[0])) continue;
-      if (softmax_block<D, BQ, BK, CAUSAL, WRITE_MASK, GAP>(p, bars, tmem, w, s, j, s ? tau1 : tau0, st, aborted) == 2)
+      if (softmax_block<D, BQ, BK, CAUSAL, WRITE_MASK, GAP, VARLEN>(p, bars, tmem, w, sp, s, j, s ? tau1 : tau0, st,
+                                                                   aborted) == 2)
         aborted = true;
     }
   }
 #pragma unroll 1
   for (int s = 0; s < 2; ++s) {
     if ((s ? w.nblk[1] : w.nblk[0]) == 0) continue;
-    softmax_epilogue<D, BQ, BK>(p, bars, tmem, w, s, st, aborted);
+    softmax_epilogue<D, BQ, BK, VARLEN>(p, bars, tmem, w, sp, s, st, aborted);
   }
 }
 
 // ---------------------------------------------------------------------------- kernel
 
-template <int D, int BQ, int BK, bool CAUSAL, bool WRITE_MASK, bool GAP>
+template <int D, int BQ, int BK, bool CAUSAL, bool WRITE_MASK, bool GAP, bool VARLEN>
 __global__ void __launch_bounds__(kThreads, 1)
     bsfa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -659,7 +695,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = smem_raw;
   Bars* bars = reinterpret_cast<Bars*>(smem + S::OFF_BAR);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const FwdUnit w = decode_unit(p, blockIdx.x, CAUSAL, BK);
+  SeqSpan sp;
+  const FwdUnit w = decode_unit<VARLEN>(p, blockIdx.x, CAUSAL, BK, sp);
+  if (VARLEN && w.nblk[0] == 0 && w.nblk[1] == 0) return;   // rows past a short packed sequence's end: no work
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
@@ -694,13 +732,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < kSoftmaxWarps) {
     regs_increase<kSoftmaxRegs>();
-    softmax_role<D, BQ, BK, CAUSAL, WRITE_MASK, GAP>(p, bars, tmem, w);
+    softmax_role<D, BQ, BK, CAUSAL, WRITE_MASK, GAP, VARLEN>(p, bars, tmem, w, sp);
   } else {
     regs_decrease<kProducerRegs>();
     if (lane == 0) {
-      if (warp == kSoftmaxWarps) kq_producer<D, BQ, BK>(&tm_q, &tm_k, smem, bars, w);
+      if (warp == kSoftmaxWarps) kq_producer<D, BQ, BK, VARLEN>(&tm_q, &tm_k, smem, bars, w, sp);
       else if (warp == kSoftmaxWarps + 1) mma_issuer<D, BQ, BK>(smem, bars, tmem, w);
-      else if (warp == kSoftmaxWarps + 2) v_producer<D, BQ, BK>(&tm_v, smem, bars, w);
+      else if (warp == kSoftmaxWarps + 2) v_producer<D, BQ, BK, VARLEN>(&tm_v, smem, bars, w, sp);
     }
     __syncwarp();
     if (warp == kSoftmaxWarps + 3) s_waiter(bars, w);

@@ -1,5 +1,5 @@
 // Kernel instantiation and launch for one head dimension (used by the per-D
-// translation units so the 64 kernel variants compile in parallel).
+// translation units so the 96 kernel variants compile in parallel).
 #pragma once
 
 #include <cuda_runtime.h>
@@ -8,11 +8,11 @@
 
 namespace bsfa {
 
-template <int D, int BQ, int BK, bool CAUSAL, bool MASK, bool GAP>
+template <int D, int BQ, int BK, bool CAUSAL, bool MASK, bool GAP, bool VARLEN = false>
 cudaError_t launch_variant(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
                            int grid, cudaStream_t stream) {
   using S = FwdShape<D, BQ, BK>;
-  auto kern = bsfa_fwd_kernel<D, BQ, BK, CAUSAL, MASK, GAP>;
+  auto kern = bsfa_fwd_kernel<D, BQ, BK, CAUSAL, MASK, GAP, VARLEN>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   kern<<<grid, kThreads, S::SMEM_BYTES, stream>>>(tq, tk, tv, p);
@@ -24,6 +24,13 @@ cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
                        int Bq, int Bk, bool causal, bool mask, int grid, cudaStream_t s) {
 #define BSFA_CASE(BQ, BK)                                                                          \
   if (Bq == BQ && Bk == BK) {                                                                      \
+    if (p.cu_seqlens != nullptr) {     /* packed sequences, threshold gate */                      \
+      if (causal)                                                                                  \
+        return mask ? launch_variant<D, BQ, BK, true, true, false, true>(tq, tk, tv, p, grid, s)   \
+                    : launch_variant<D, BQ, BK, true, false, false, true>(tq, tk, tv, p, grid, s); \
+      return mask ? launch_variant<D, BQ, BK, false, true, false, true>(tq, tk, tv, p, grid, s)    \
+                  : launch_variant<D, BQ, BK, false, false, false, true>(tq, tk, tv, p, grid, s);  \
+    }                                                                                              \
     if (p.gate_gap) {                                                                              \
       if (causal)                                                                                  \
         return mask ? launch_variant<D, BQ, BK, true, true, true>(tq, tk, tv, p, grid, s)          \
