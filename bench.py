@@ -159,8 +159,11 @@ def kernel_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def measured_traffic(cfg):
-    """DRAM bytes per launch from the committed ncu summary, if it matches this kernel and workload."""
+def measured_traffic(cfg, tau_desc):
+    """DRAM bytes per launch from the committed ncu summary, if it matches this kernel and workload
+    (the per-head threshold gate it was captured with)."""
+    if tau_desc.get("tau") != "per head":
+        return None
     if not os.path.exists(TRAFFIC):
         return None
     kv = {}
@@ -391,7 +394,7 @@ def run_ours(args):
             peaks = json.load(f)
         if peaks.get("bf16_tflops"):
             peak, peak_src = float(peaks["bf16_tflops"]), "measured (MEASURED_PEAKS.json bf16_tflops, burst)"
-    traffic = measured_traffic(cfg)
+    traffic = measured_traffic(cfg, p)
 
     line = None
     if rank == 0:
