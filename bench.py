@@ -65,6 +65,9 @@ def parse():
     ap.add_argument("--gate", choices=["tau", "gap"], default="tau",
                     help="tau: the BSFA gate; gap: the gap-to-running-maximum gate, for comparison")
     ap.add_argument("--gamma", type=float, default=-1.0, help="gamma of the gap gate (scaled-score units)")
+    ap.add_argument("--shard", choices=["replica", "heads"], default="replica",
+                    help="multi-GPU layout: replica = every rank runs the whole layer (weak scaling); heads = the "
+                         "layer's KV groups are split across the ranks (strong scaling, no exchange needed)")
     ap.add_argument("--curve", action="store_true",
                     help="instead of the bench line: error against dense attention, skip fraction and time for "
                          "several settings of each gate (one JSON line each)")
@@ -134,6 +137,15 @@ def oracle_sample(cfg, x, taus, budget_s, tiles, gate="tau"):
         if time.perf_counter() - t0 >= budget_s:
             break
     return flops, time.perf_counter() - t0, done
+
+
+def head_shard(rank: int, world: int, Hkv: int) -> tuple[int, int]:
+    """(first KV head, KV head count) of ``rank`` when a layer's KV groups are split
+    evenly across ``world`` ranks."""
+    if Hkv % world != 0:
+        raise ValueError(f"{Hkv} KV heads do not split evenly across {world} ranks")
+    per = Hkv // world
+    return rank * per, per
 
 
 def max_over_ranks(value: float, dist=None, device=None) -> float:
@@ -282,6 +294,10 @@ def run_ours(args):
     bsfa.load()
 
     cfg, p, taus = workload(args)
+    heads = args.shard == "heads"
+    if heads and (args.gate != "tau" or args.tau_table is not None):
+        raise SystemExit("--shard heads runs the per-head threshold gate only")
+    kv_begin, kv_count = head_shard(rank, world, cfg.Hkv) if heads else (0, cfg.Hkv)
     x = make_inputs(cfg)
     to_dev = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
     q, k, v = to_dev(x["q"]), to_dev(x["k"]), to_dev(x["v"])
@@ -293,7 +309,10 @@ def run_ours(args):
     stream = torch.cuda.current_stream(dev)
 
     def step(t):
-        if args.gate == "gap" and t is not tau_dense:
+        if heads:
+            st = bsfa.bsfa_forward_heads(q, k, v, t, out, lse, None, cfg.B, cfg.Hq, cfg.Hkv, cfg.N, cfg.D, cfg.Bq,
+                                         cfg.Bk, cfg.causal, kv_begin, kv_count, stream)
+        elif args.gate == "gap" and t is not tau_dense:
             st = bsfa.bsfa_forward_gap(q, k, v, t, out, lse, None, cfg.B, cfg.Hq, cfg.Hkv, cfg.N, cfg.D, cfg.Bq, cfg.Bk,
                                        cfg.causal, stream)
         elif t.dim() == 1:
@@ -310,6 +329,9 @@ def run_ours(args):
                               gate=args.gate)
     m = mask.cpu().numpy()
     del mask
+    layer_dense_flops = mask_flops(m, cfg)[1]
+    g = cfg.Hq // cfg.Hkv
+    m = m[:, kv_begin * g:(kv_begin + kv_count) * g]      # this rank's heads (all of them unless head-sharded)
     exec_flops, dense_flops = mask_flops(m, cfg)
     gated = np.isin(m, (0, 1))
     achieved_skip = float((m == 0).sum() / max(gated.sum(), 1))
@@ -353,7 +375,7 @@ def run_ours(args):
     dense_ms = max_over_ranks(sum(timed(tau_dense, args.steps)), dist, dev) / args.steps
 
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not heads:
         hq = torch.empty(q.shape, dtype=torch.bfloat16, pin_memory=True)
         hk = torch.empty(k.shape, dtype=torch.bfloat16, pin_memory=True)
         hv = torch.empty(v.shape, dtype=torch.bfloat16, pin_memory=True)
@@ -399,11 +421,14 @@ def run_ours(args):
     line = None
     if rank == 0:
         line = {
-            "metric": METRIC, "value": weak_scaling_value(dense_flops, world, ms), "unit": UNIT, "n_gpus": world,
-            "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "metric": METRIC,
+            "value": layer_dense_flops / (ms * 1e-3) / 1e12 if heads else weak_scaling_value(dense_flops, world, ms),
+            "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "strong" if heads else "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": config_record(cfg, p, achieved_skip),
+            "config": {**config_record(cfg, p, achieved_skip),
+                       **({"parallelism": f"KV heads split across {world} GPUs"} if heads else {})},
             "exec_tflops": world * exec_tflops, "dense_equiv_tflops": world * dense_tflops,
             "ms_per_layer": ms, "dense_ms_per_layer": dense_ms, "speedup_vs_dense": dense_ms / ms,
             "exec_flops_per_layer": exec_flops, "dense_flops_per_layer": dense_flops,

@@ -118,6 +118,20 @@ bsfa_status bsfa_forward_gap(const void* q, const void* k, const void* v, const 
                              void* stream);
 
 /*
+ * bsfa_forward_heads - bsfa_forward for the query heads of KV heads
+ * [kv_begin, kv_begin + kv_count) only: one head shard of the layer, for
+ * splitting a layer's KV groups across GPUs. Heads are independent problems,
+ * so the shards need no exchange. All tensors keep their full [.., Hq or Hkv, ..]
+ * shapes and strides; only the selected heads' rows of out and lse are written.
+ * The block mask, if given, is filled with 3 whole, then written for the
+ * selected heads. 0 <= kv_begin, 1 <= kv_count, kv_begin + kv_count <= Hkv,
+ * else BSFA_ERR_INVALID_ARG; everything else as bsfa_forward.
+ */
+bsfa_status bsfa_forward_heads(const void* q, const void* k, const void* v, const float* tau, void* out, float* lse,
+                               uint8_t* block_mask, int B, int Hq, int Hkv, int N, int D, int Bq, int Bk, int causal,
+                               int kv_begin, int kv_count, void* stream);
+
+/*
  * bsfa_forward_varlen - bsfa_forward over a packed batch of sequences of
  * different lengths (mixed-length prefill). Sequence e holds rows
  * [cu_seqlens[e], cu_seqlens[e+1]) of the packed tensors; each sequence is its

@@ -97,3 +97,11 @@ def test_varlen_entry_rejects_bad_arguments_without_touching_cuda(lib):
     assert call(18, 2, 500) == bsfa.BSFA_ERR_INVALID_ARG            # misaligned offsets
     assert call(16, 2, 4097 * 128) == bsfa.BSFA_ERR_UNSUPPORTED     # too many key blocks
     assert call(16, 2, 500, D=96) == bsfa.BSFA_ERR_UNSUPPORTED      # head dimension
+
+
+def test_head_shard_entry_rejects_bad_ranges_without_touching_cuda(lib):
+    call = lambda b, c: bsfa.bsfa_forward_heads(16, 16, 16, 16, 16, None, None, 1, 8, 4, 512, 128, 128, 128, 1, b, c,
+                                                None)
+    for b, c in ((-1, 2), (0, 0), (0, -1), (3, 2), (4, 1)):
+        assert call(b, c) == bsfa.BSFA_ERR_INVALID_ARG, (b, c)
+        assert "kv" in bsfa.bsfa_last_error().lower() or "heads" in bsfa.bsfa_last_error()

@@ -189,3 +189,33 @@ def test_gap_gate_on_the_8k_layer():
     stats["skip_fraction"] = float((m == 0).sum() / max(np.isin(m, (0, 1)).sum(), 1))
     print("c2 gap", stats)
     assert 0.2 < stats["skip_fraction"] < 0.95
+
+
+# ----------------------------------------------------------------------------- head shards
+
+@pytest.mark.parametrize("Hq,Hkv,shards", [(8, 4, 2), (8, 4, 4), (6, 6, 3)])
+def test_head_shards_equal_the_whole_layer(Hq, Hkv, shards):
+    """Each shard (bsfa_forward_heads) writes exactly its heads, bit for bit what the
+    whole-layer call writes for them; other heads are left as they were."""
+    cfg, x = _inputs(1000, 128, Hq, Hkv, 128, 128, True, kind="planted", seed=60 + shards)
+    tau = calibrate(x["q"], x["k"], 128, 128, True, [0.5])[0.5]
+    whole = run_gpu(x, tau, 128, 128, True)
+    from parity import to_device
+    q, k, v = (to_device(x[n]) for n in "qkv")
+    t = torch.tensor(np.asarray(tau, dtype=np.float32), device="cuda")
+    out = torch.full_like(q, 7.0)
+    lse = torch.full((1, Hq, 1000), 7.0, dtype=torch.float32, device="cuda")
+    per = Hkv // shards
+    g = Hq // Hkv
+    for s in range(shards):
+        assert bsfa.bsfa_forward_heads(q, k, v, t, out, lse, None, 1, Hq, Hkv, 1000, 128, 128, 128, True, s * per, per,
+                                       None) == bsfa.BSFA_OK
+        torch.cuda.synchronize()
+        o = out.float().cpu().numpy()
+        l = lse.cpu().numpy()
+        done = slice(0, (s + 1) * per * g)
+        assert np.array_equal(o[:, :, done], whole["out"][:, :, done])
+        assert np.array_equal(l[:, done], whole["lse"][:, done])
+        if s + 1 < shards:
+            assert (o[:, :, (s + 1) * per * g:] == 7.0).all()
+    assert bsfa.bsfa_get_status(None) == bsfa.BSFA_OK

@@ -1,9 +1,10 @@
 """The N > 1 path on the CPU: world-size-2 gloo process groups.
 
 bench.py runs one rank per GPU with no data-path collective (every rank owns an
-independent layer); the only cross-rank steps are the barrier and the
-max-over-ranks reduction of the timed region. These tests run that reduction and
-the reference arm's rank handling with two gloo ranks.
+independent layer, or with --shard heads a disjoint run of the layer's KV
+heads); the only cross-rank steps are the barrier and the max-over-ranks
+reduction of the timed region. These tests run that reduction, the head-shard
+assignment and the reference arm's rank handling with two gloo ranks.
 """
 import json
 import os
@@ -49,6 +50,42 @@ def test_max_over_ranks_and_weak_scaling_with_two_gloo_ranks():
     assert [r[1] for r in results] == [15.0, 15.0]            # every rank sees the slowest rank's time
     for _, _, value in results:
         assert abs(value - 2 * 1.0e12 / 15e-3 / 1e12) < 1e-9     # both ranks' FLOPs over the slowest time
+
+
+def _shard_main(rank, world, port, queue):
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    import torch
+    import torch.distributed as dist
+    import bench
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    begin, count = bench.head_shard(rank, world, 8)
+    mine = torch.tensor([begin, count])
+    every = [torch.zeros(2, dtype=mine.dtype) for _ in range(world)]
+    dist.all_gather(every, mine)
+    queue.put((rank, [tuple(t.tolist()) for t in every]))
+    dist.destroy_process_group()
+
+
+def test_head_shards_cover_the_kv_heads_once_with_two_gloo_ranks():
+    """--shard heads: each rank takes a disjoint run of KV heads; together all of them."""
+    ctx = mp.get_context("spawn")
+    queue = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_shard_main, args=(r, 2, port, queue)) for r in range(2)]
+    for p in procs:
+        p.start()
+    results = sorted(queue.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for _, shards in results:
+        assert shards == [(0, 4), (4, 4)]
+    sys.path.insert(0, ROOT)
+    import bench
+    import pytest
+    with pytest.raises(ValueError):
+        bench.head_shard(0, 3, 8)
 
 
 def test_single_process_needs_no_group():

@@ -6,7 +6,7 @@ fallback: if the library is missing or the device is not sm_100, calls fail
 loudly.
 
 The functions named like the C entry points (``bsfa_forward``,
-``bsfa_forward_tau_table``, ``bsfa_forward_gap``, ``bsfa_forward_varlen``, ``bsfa_validate``,
+``bsfa_forward_tau_table``, ``bsfa_forward_gap``, ``bsfa_forward_heads``, ``bsfa_forward_varlen``, ``bsfa_validate``,
 ``bsfa_get_status``,
 ``bsfa_selftest_lost_arrival``, ``bsfa_status_string``, ``bsfa_last_error``)
 take the same arguments; pointer arguments accept an int
@@ -27,9 +27,9 @@ BSFA_ERR_UNSUPPORTED = 2
 BSFA_ERR_CUDA = 3
 BSFA_ERR_DEVICE_TIMEOUT = 4
 
-EXPORTED = ("bsfa_forward", "bsfa_forward_tau_table", "bsfa_forward_gap", "bsfa_forward_varlen", "bsfa_validate",
-            "bsfa_get_status",
-            "bsfa_selftest_lost_arrival", "bsfa_status_string", "bsfa_last_error")
+EXPORTED = ("bsfa_forward", "bsfa_forward_tau_table", "bsfa_forward_gap", "bsfa_forward_heads", "bsfa_forward_varlen",
+            "bsfa_validate", "bsfa_get_status", "bsfa_selftest_lost_arrival", "bsfa_status_string",
+            "bsfa_last_error")
 
 _lib = None
 
@@ -55,6 +55,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.bsfa_forward_tau_table.restype = i
     lib.bsfa_forward_gap.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, vp]
     lib.bsfa_forward_gap.restype = i
+    lib.bsfa_forward_heads.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, i, vp]
+    lib.bsfa_forward_heads.restype = i
     lib.bsfa_forward_varlen.argtypes = [vp, vp, vp, vp, i, i, vp, vp, vp, vp, i, i, i, i, i, i, i, vp]
     lib.bsfa_forward_varlen.restype = i
     lib.bsfa_validate.argtypes = [i] * 8
@@ -104,6 +106,13 @@ def bsfa_forward_tau_table(q, k, v, tau_table, tau_tiles, out, lse, block_mask, 
 def bsfa_forward_gap(q, k, v, gamma, out, lse, block_mask, B, Hq, Hkv, N, D, Bq, Bk, causal, stream) -> int:
     return load().bsfa_forward_gap(_ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(out), _ptr(lse), _ptr(block_mask),
                                    B, Hq, Hkv, N, D, Bq, Bk, int(bool(causal)), _stream(stream))
+
+
+def bsfa_forward_heads(q, k, v, tau, out, lse, block_mask, B, Hq, Hkv, N, D, Bq, Bk, causal, kv_begin, kv_count,
+                       stream) -> int:
+    return load().bsfa_forward_heads(_ptr(q), _ptr(k), _ptr(v), _ptr(tau), _ptr(out), _ptr(lse), _ptr(block_mask),
+                                     B, Hq, Hkv, N, D, Bq, Bk, int(bool(causal)), int(kv_begin), int(kv_count),
+                                     _stream(stream))
 
 
 def bsfa_forward_varlen(q, k, v, cu_seqlens, nseq, max_seqlen, tau, out, lse, block_mask, total, Hq, Hkv, D, Bq, Bk,

@@ -132,7 +132,8 @@ namespace {
 // packed sequences of at most max_seqlen rows in N = total rows.
 bsfa_status forward_impl(const void* q, const void* k, const void* v, const float* tau, int tau_tiles, int gate_gap,
                          void* out, float* lse, uint8_t* block_mask, int B, int Hq, int Hkv, int N, int D, int Bq,
-                         int Bk, int causal, void* stream, const int* cu_seqlens = nullptr, int max_seqlen = 0) {
+                         int Bk, int causal, void* stream, const int* cu_seqlens = nullptr, int max_seqlen = 0,
+                         int kv_begin = 0, int kv_count = -1) {
   bsfa_status st = cu_seqlens ? bsfa_validate(1, Hq, Hkv, N, D, Bq, Bk, causal)
                               : bsfa_validate(B, Hq, Hkv, N, D, Bq, Bk, causal);
   if (st != BSFA_OK) return st;
@@ -147,6 +148,9 @@ bsfa_status forward_impl(const void* q, const void* k, const void* v, const floa
   } else {
     max_seqlen = N;
   }
+  if (kv_count < 0) kv_count = Hkv;
+  if (kv_begin < 0 || kv_count <= 0 || kv_begin + kv_count > Hkv)
+    return fail(BSFA_ERR_INVALID_ARG, "KV heads [%d, %d) are not inside [0, %d)", kv_begin, kv_begin + kv_count, Hkv);
   if (tau_tiles < 0) return fail(BSFA_ERR_INVALID_ARG, "tau_tiles=%d is negative", tau_tiles);
   if (!q || !k || !v || !tau || !out) return fail(BSFA_ERR_INVALID_ARG, "q, k, v, tau and out must be non-null");
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16))
@@ -193,10 +197,12 @@ bsfa_status forward_impl(const void* q, const void* k, const void* v, const floa
   // A CTA pairs two query heads of one KV group when the group size is even,
   // otherwise two adjacent 128-row tiles of one head.
   p.pair_heads = (p.group % 2 == 0) ? 1 : 0;
+  p.hq_begin = kv_begin * p.group;
+  p.hq_count = kv_count * p.group;
   p.scale = (float)(1.0 / std::sqrt((double)D));
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
   const int tiles = (max_seqlen + 127) / 128;
-  const int grid = p.pair_heads ? B * (Hq / 2) * tiles : B * Hq * ((tiles + 1) / 2);
+  const int grid = p.pair_heads ? B * (p.hq_count / 2) * tiles : B * p.hq_count * ((tiles + 1) / 2);
   e = (D == 64) ? bsfa::launch_fwd_d64(tq, tk, tv, p, Bq, Bk, causal != 0, block_mask != nullptr, grid, s)
                 : bsfa::launch_fwd_d128(tq, tk, tv, p, Bq, Bk, causal != 0, block_mask != nullptr, grid, s);
   if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
@@ -225,6 +231,16 @@ bsfa_status bsfa_forward_gap(const void* q, const void* k, const void* v, const 
                              uint8_t* block_mask, int B, int Hq, int Hkv, int N, int D, int Bq, int Bk, int causal,
                              void* stream) {
   return forward_impl(q, k, v, gamma, 0, 1, out, lse, block_mask, B, Hq, Hkv, N, D, Bq, Bk, causal, stream);
+}
+
+bsfa_status bsfa_forward_heads(const void* q, const void* k, const void* v, const float* tau, void* out, float* lse,
+                               uint8_t* block_mask, int B, int Hq, int Hkv, int N, int D, int Bq, int Bk, int causal,
+                               int kv_begin, int kv_count, void* stream) {
+  if (kv_begin < 0 || kv_count < 1)
+    return fail(BSFA_ERR_INVALID_ARG, "kv_begin=%d, kv_count=%d: need kv_begin >= 0 and kv_count >= 1", kv_begin,
+                kv_count);
+  return forward_impl(q, k, v, tau, 0, 0, out, lse, block_mask, B, Hq, Hkv, N, D, Bq, Bk, causal, stream, nullptr, 0,
+                      kv_begin, kv_count);
 }
 
 bsfa_status bsfa_forward_varlen(const void* q, const void* k, const void* v, const int* cu_seqlens, int nseq,

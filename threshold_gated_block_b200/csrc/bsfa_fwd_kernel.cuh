@@ -51,6 +51,7 @@ struct FwdParams {
   int max_seqlen;     // longest sequence (N for [B, N] inputs): sizes the grid
   int mask_mq, mask_mkv;   // query tiles and key blocks per sequence in the block mask
   int group;          // Hq / Hkv
+  int hq_begin, hq_count;   // the query heads this launch computes (all of them unless head-sharded)
   int pair_heads;     // 1: slots are query heads 2p and 2p+1 on the same rows
   int gate_gap;       // 0: the BSFA gate (block maximum against tau); 1: the gap gate, tau holding gamma
                       // (selects the kernel's GAP template argument at launch)
@@ -138,21 +139,21 @@ __device__ __forceinline__ FwdUnit decode_unit(const FwdParams& p, int u, bool c
   FwdUnit w;
   if (p.pair_heads) {
     // Consecutive units: the head pairs of one row block, a KV group's pairs adjacent.
-    const int per = p.B * (p.Hq / 2);
+    const int per = p.B * (p.hq_count / 2);
     const int hp = u % per, t = u / per;
     const int qt = causal ? tiles - 1 - t : t;     // heaviest causal rows first
-    w.b = hp / (p.Hq / 2);
-    const int h0 = 2 * (hp % (p.Hq / 2));
+    w.b = hp / (p.hq_count / 2);
+    const int h0 = p.hq_begin + 2 * (hp % (p.hq_count / 2));
     w.hq[0] = h0;
     w.hq[1] = h0 + 1;
     w.q0[0] = w.q0[1] = qt * 128;
   } else {
     const int pairs = (tiles + 1) / 2;
-    const int per = p.B * p.Hq;
+    const int per = p.B * p.hq_count;
     const int bh = u % per, t = u / per;
     const int qp = causal ? pairs - 1 - t : t;
-    w.b = bh / p.Hq;
-    w.hq[0] = w.hq[1] = bh % p.Hq;
+    w.b = bh / p.hq_count;
+    w.hq[0] = w.hq[1] = p.hq_begin + bh % p.hq_count;
     w.q0[0] = 2 * qp * 128;
     w.q0[1] = w.q0[0] + 128;
   }
