@@ -24,7 +24,8 @@
  *
  * Thread safety: entry points may be called from several host threads; calls on
  * the same stream are ordered by the stream. The library allocates nothing per
- * call; it keeps one device status word per device.
+ * call; it keeps one device status word per device (and, for bsfa_forward_host,
+ * two copy streams and their events per device, created on first use).
  */
 #ifndef BSFA_H_
 #define BSFA_H_
@@ -130,6 +131,32 @@ bsfa_status bsfa_forward_gap(const void* q, const void* k, const void* v, const 
 bsfa_status bsfa_forward_heads(const void* q, const void* k, const void* v, const float* tau, void* out, float* lse,
                                uint8_t* block_mask, int B, int Hq, int Hkv, int N, int D, int Bq, int Bk, int causal,
                                int kv_begin, int kv_count, void* stream);
+
+/*
+ * bsfa_forward_host - bsfa_forward on HOST buffers, with the copies overlapped
+ * with the kernel: the layer is cut into `chunks` runs of KV heads (as even as
+ * Hkv allows); chunk c's Q/K/V go up on a copy stream, its heads are computed
+ * (bsfa_forward_heads) once they have landed, and its out/lse rows come back on a
+ * second copy stream while the next chunk computes. Asynchronous: everything is
+ * done once `stream` reaches the call.
+ *
+ *   q_host, k_host, v_host, tau_host   inputs in host memory, the layouts of
+ *                                      bsfa_forward; page-locked (pinned) memory is
+ *                                      needed for the copies to overlap
+ *   out_host, lse_host                 results in host memory (lse_host may be NULL)
+ *   q_dev ... lse_dev                  device buffers of bsfa_forward's shapes, owned
+ *                                      by the caller (lse_dev NULL iff lse_host is)
+ *   chunks                             1 <= chunks <= min(Hkv, 64)
+ *
+ * The library creates two copy streams and their events once per device and
+ * reuses them; calls on one device share them (their copies are serialised).
+ * Errors as bsfa_forward; BSFA_ERR_INVALID_ARG for a bad chunk count or a
+ * missing buffer.
+ */
+bsfa_status bsfa_forward_host(const void* q_host, const void* k_host, const void* v_host, const float* tau_host,
+                              void* out_host, float* lse_host, void* q_dev, void* k_dev, void* v_dev, float* tau_dev,
+                              void* out_dev, float* lse_dev, int B, int Hq, int Hkv, int N, int D, int Bq, int Bk,
+                              int causal, int chunks, void* stream);
 
 /*
  * bsfa_forward_varlen - bsfa_forward over a packed batch of sequences of

@@ -105,3 +105,17 @@ def test_head_shard_entry_rejects_bad_ranges_without_touching_cuda(lib):
     for b, c in ((-1, 2), (0, 0), (0, -1), (3, 2), (4, 1)):
         assert call(b, c) == bsfa.BSFA_ERR_INVALID_ARG, (b, c)
         assert "kv" in bsfa.bsfa_last_error().lower() or "heads" in bsfa.bsfa_last_error()
+
+
+def test_host_buffer_entry_rejects_bad_arguments_without_touching_cuda(lib):
+    ptrs = [16] * 12
+    shape = (1, 8, 4, 512, 128, 128, 128, 1)
+    assert bsfa.bsfa_forward_host(*ptrs, *shape, 0, None) == bsfa.BSFA_ERR_INVALID_ARG        # no chunks
+    assert bsfa.bsfa_forward_host(*ptrs, *shape, 5, None) == bsfa.BSFA_ERR_INVALID_ARG        # more chunks than KV heads
+    missing = list(ptrs)
+    missing[6] = None                                                                          # no device q
+    assert bsfa.bsfa_forward_host(*missing, *shape, 2, None) == bsfa.BSFA_ERR_INVALID_ARG
+    half_lse = list(ptrs)
+    half_lse[11] = None                                                                        # lse on one side only
+    assert bsfa.bsfa_forward_host(*half_lse, *shape, 2, None) == bsfa.BSFA_ERR_INVALID_ARG
+    assert bsfa.bsfa_forward_host(*ptrs, 1, 8, 4, 512, 96, 128, 128, 1, 2, None) == bsfa.BSFA_ERR_UNSUPPORTED

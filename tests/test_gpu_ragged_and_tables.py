@@ -219,3 +219,22 @@ def test_head_shards_equal_the_whole_layer(Hq, Hkv, shards):
         if s + 1 < shards:
             assert (o[:, :, (s + 1) * per * g:] == 7.0).all()
     assert bsfa.bsfa_get_status(None) == bsfa.BSFA_OK
+
+
+# ----------------------------------------------------------------------------- host buffers, overlapped copies
+
+@pytest.mark.parametrize("chunks", [1, 3, 4])
+def test_host_buffer_call_equals_the_device_call(chunks):
+    """bsfa_forward_host (copies in runs of KV heads, overlapped with the kernel)
+    returns exactly what the device call computes, for an uneven chunk split and a
+    ragged N."""
+    cfg, x = _inputs(900, 128, 8, 4, 128, 64, True, kind="planted", seed=70)
+    tau = calibrate(x["q"], x["k"], 128, 64, True, [0.5])[0.5]
+    dev = run_gpu(x, tau, 128, 64, True, want_mask=False)
+    host = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).pin_memory()
+    q, k, v = (host(x[n]) for n in "qkv")
+    t = torch.tensor(np.asarray(tau, dtype=np.float32)).pin_memory()
+    out, lse = bsfa.forward_host(q, k, v, t, Bq=128, Bk=64, causal=True, chunks=chunks)
+    assert bsfa.bsfa_get_status(None) == bsfa.BSFA_OK
+    assert np.array_equal(out.float().numpy().astype(np.float64), dev["out"])
+    assert np.array_equal(lse.numpy().astype(np.float64), dev["lse"])

@@ -6,7 +6,8 @@ fallback: if the library is missing or the device is not sm_100, calls fail
 loudly.
 
 The functions named like the C entry points (``bsfa_forward``,
-``bsfa_forward_tau_table``, ``bsfa_forward_gap``, ``bsfa_forward_heads``, ``bsfa_forward_varlen``, ``bsfa_validate``,
+``bsfa_forward_tau_table``, ``bsfa_forward_gap``, ``bsfa_forward_heads``, ``bsfa_forward_host``,
+``bsfa_forward_varlen``, ``bsfa_validate``,
 ``bsfa_get_status``,
 ``bsfa_selftest_lost_arrival``, ``bsfa_status_string``, ``bsfa_last_error``)
 take the same arguments; pointer arguments accept an int
@@ -27,9 +28,9 @@ BSFA_ERR_UNSUPPORTED = 2
 BSFA_ERR_CUDA = 3
 BSFA_ERR_DEVICE_TIMEOUT = 4
 
-EXPORTED = ("bsfa_forward", "bsfa_forward_tau_table", "bsfa_forward_gap", "bsfa_forward_heads", "bsfa_forward_varlen",
-            "bsfa_validate", "bsfa_get_status", "bsfa_selftest_lost_arrival", "bsfa_status_string",
-            "bsfa_last_error")
+EXPORTED = ("bsfa_forward", "bsfa_forward_tau_table", "bsfa_forward_gap", "bsfa_forward_heads", "bsfa_forward_host",
+            "bsfa_forward_varlen", "bsfa_validate", "bsfa_get_status", "bsfa_selftest_lost_arrival",
+            "bsfa_status_string", "bsfa_last_error")
 
 _lib = None
 
@@ -57,6 +58,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.bsfa_forward_gap.restype = i
     lib.bsfa_forward_heads.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, i, vp]
     lib.bsfa_forward_heads.restype = i
+    lib.bsfa_forward_host.argtypes = [vp] * 12 + [i] * 9 + [vp]
+    lib.bsfa_forward_host.restype = i
     lib.bsfa_forward_varlen.argtypes = [vp, vp, vp, vp, i, i, vp, vp, vp, vp, i, i, i, i, i, i, i, vp]
     lib.bsfa_forward_varlen.restype = i
     lib.bsfa_validate.argtypes = [i] * 8
@@ -113,6 +116,13 @@ def bsfa_forward_heads(q, k, v, tau, out, lse, block_mask, B, Hq, Hkv, N, D, Bq,
     return load().bsfa_forward_heads(_ptr(q), _ptr(k), _ptr(v), _ptr(tau), _ptr(out), _ptr(lse), _ptr(block_mask),
                                      B, Hq, Hkv, N, D, Bq, Bk, int(bool(causal)), int(kv_begin), int(kv_count),
                                      _stream(stream))
+
+
+def bsfa_forward_host(q_host, k_host, v_host, tau_host, out_host, lse_host, q_dev, k_dev, v_dev, tau_dev, out_dev,
+                      lse_dev, B, Hq, Hkv, N, D, Bq, Bk, causal, chunks, stream) -> int:
+    return load().bsfa_forward_host(*(_ptr(t) for t in (q_host, k_host, v_host, tau_host, out_host, lse_host, q_dev,
+                                                        k_dev, v_dev, tau_dev, out_dev, lse_dev)),
+                                    B, Hq, Hkv, N, D, Bq, Bk, int(bool(causal)), int(chunks), _stream(stream))
 
 
 def bsfa_forward_varlen(q, k, v, cu_seqlens, nseq, max_seqlen, tau, out, lse, block_mask, total, Hq, Hkv, D, Bq, Bk,
@@ -219,11 +229,14 @@ def forward_varlen(q, k, v, cu_seqlens, max_seqlen: int, tau, *, Bq: int, Bk: in
 
 
 def forward_host(q, k, v, tau, *, Bq: int, Bk: int, causal: bool, device=None, stream=None, bufs=None,
-                 gate: str = "tau"):
+                 gate: str = "tau", chunks: int | None = None):
     """End-to-end call on host tensors: copy inputs to the device, run, copy out and lse back.
 
     q, k, v: bf16 CPU tensors (pinned for asynchronous copies); tau: fp32 CPU tensor, [Hq] or [Hq, T].
     ``bufs`` (from ``device_buffers``) holds reusable device and pinned host buffers.
+    With one threshold per head this is ``bsfa_forward_host``: the copies run in
+    ``chunks`` runs of KV heads (default min(Hkv, 8)) overlapped with the kernel.
+    Other gates copy, run and copy back in turn on ``stream``.
     Returns (out_host, lse_host).
     """
     import torch
@@ -232,6 +245,14 @@ def forward_host(q, k, v, tau, *, Bq: int, Bk: int, causal: bool, device=None, s
         stream = torch.cuda.current_stream(device)
     if bufs is None:
         bufs = device_buffers(q.shape, k.shape, device, tuple(tau.shape))
+    if gate == "tau" and tau.dim() == 1:
+        B, N, Hq, D = q.shape
+        Hkv = k.shape[2]
+        _check(bsfa_forward_host(q, k, v, tau, bufs["out_host"], bufs["lse_host"], bufs["q"], bufs["k"], bufs["v"],
+                                 bufs["tau"], bufs["out"], bufs["lse"], B, Hq, Hkv, N, D, Bq, Bk, causal,
+                                 chunks or min(Hkv, 8), stream))
+        stream.synchronize()
+        return bufs["out_host"], bufs["lse_host"]
     with torch.cuda.stream(stream):
         for name, src in (("q", q), ("k", k), ("v", v), ("tau", tau)):
             bufs[name].copy_(src, non_blocking=True)

@@ -209,6 +209,47 @@ bsfa_status forward_impl(const void* q, const void* k, const void* v, const floa
   return BSFA_OK;
 }
 
+// Copy streams and events of the host-buffer path, created once per device and
+// reused by every call (so a call allocates nothing). Calls on one device share
+// them, which orders (and serialises) their copies.
+constexpr int kMaxChunks = 64;
+struct HostPipe {
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t start = nullptr, in[kMaxChunks] = {}, done[kMaxChunks] = {}, out = nullptr;
+};
+HostPipe g_pipe[kMaxDevices];
+std::mutex g_pipe_mutex;
+
+bsfa_status host_pipe(int dev, HostPipe** pipe) {
+  std::lock_guard<std::mutex> lock(g_pipe_mutex);
+  HostPipe& hp = g_pipe[dev];
+  if (hp.h2d == nullptr) {
+    cudaError_t e = cudaStreamCreateWithFlags(&hp.h2d, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&hp.d2h, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&hp.start, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&hp.out, cudaEventDisableTiming);
+    for (int c = 0; c < kMaxChunks && e == cudaSuccess; ++c) {
+      e = cudaEventCreateWithFlags(&hp.in[c], cudaEventDisableTiming);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&hp.done[c], cudaEventDisableTiming);
+    }
+    if (e != cudaSuccess) {
+      hp.h2d = nullptr;
+      return cuda_fail(e, "creating the copy streams");
+    }
+  }
+  *pipe = &hp;
+  return BSFA_OK;
+}
+
+// Rows [0, rows) of a row-major [rows, cols_total] array of `elem`-byte
+// elements, columns [col0, col0 + cols): one strided copy.
+cudaError_t copy_cols(void* dst, const void* src, size_t rows, size_t cols_total, size_t col0, size_t cols, size_t elem,
+                      cudaMemcpyKind kind, cudaStream_t st) {
+  const size_t pitch = cols_total * elem;
+  return cudaMemcpy2DAsync(static_cast<char*>(dst) + col0 * elem, pitch, static_cast<const char*>(src) + col0 * elem,
+                           pitch, cols * elem, rows, kind, st);
+}
+
 }  // namespace
 
 extern "C" {
@@ -241,6 +282,67 @@ bsfa_status bsfa_forward_heads(const void* q, const void* k, const void* v, cons
                 kv_count);
   return forward_impl(q, k, v, tau, 0, 0, out, lse, block_mask, B, Hq, Hkv, N, D, Bq, Bk, causal, stream, nullptr, 0,
                       kv_begin, kv_count);
+}
+
+bsfa_status bsfa_forward_host(const void* q_host, const void* k_host, const void* v_host, const float* tau_host,
+                              void* out_host, float* lse_host, void* q_dev, void* k_dev, void* v_dev, float* tau_dev,
+                              void* out_dev, float* lse_dev, int B, int Hq, int Hkv, int N, int D, int Bq, int Bk,
+                              int causal, int chunks, void* stream) {
+  bsfa_status st = bsfa_validate(B, Hq, Hkv, N, D, Bq, Bk, causal);
+  if (st != BSFA_OK) return st;
+  if (!q_host || !k_host || !v_host || !tau_host || !out_host || !q_dev || !k_dev || !v_dev || !tau_dev || !out_dev)
+    return fail(BSFA_ERR_INVALID_ARG, "host and device q, k, v, tau and out must be non-null");
+  if ((lse_host == nullptr) != (lse_dev == nullptr))
+    return fail(BSFA_ERR_INVALID_ARG, "lse needs both a host and a device buffer, or neither");
+  if (chunks < 1 || chunks > Hkv || chunks > kMaxChunks)
+    return fail(BSFA_ERR_INVALID_ARG, "chunks=%d must be in [1, min(Hkv=%d, %d)]", chunks, Hkv, kMaxChunks);
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(BSFA_ERR_UNSUPPORTED, "device index %d out of range", dev);
+  HostPipe* hp = nullptr;
+  st = host_pipe(dev, &hp);
+  if (st != BSFA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int group = Hq / Hkv;
+  const size_t rows = (size_t)B * N;
+  // The copies start once earlier work on the caller's stream is done.
+  e = cudaEventRecord(hp->start, s);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(hp->h2d, hp->start, 0);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(tau_dev, tau_host, (size_t)Hq * sizeof(float), cudaMemcpyHostToDevice, hp->h2d);
+  if (e != cudaSuccess) return cuda_fail(e, "host pipeline start");
+  for (int c = 0; c < chunks; ++c) {
+    // Chunk c: KV heads [g0, g1) and their query heads, as even a split as Hkv allows.
+    const int g0 = (int)((long long)Hkv * c / chunks), g1 = (int)((long long)Hkv * (c + 1) / chunks);
+    const int h0 = g0 * group, nh = (g1 - g0) * group;
+    e = copy_cols(q_dev, q_host, rows, (size_t)Hq * D, (size_t)h0 * D, (size_t)nh * D, 2, cudaMemcpyHostToDevice, hp->h2d);
+    if (e == cudaSuccess)
+      e = copy_cols(k_dev, k_host, rows, (size_t)Hkv * D, (size_t)g0 * D, (size_t)(g1 - g0) * D, 2,
+                    cudaMemcpyHostToDevice, hp->h2d);
+    if (e == cudaSuccess)
+      e = copy_cols(v_dev, v_host, rows, (size_t)Hkv * D, (size_t)g0 * D, (size_t)(g1 - g0) * D, 2,
+                    cudaMemcpyHostToDevice, hp->h2d);
+    if (e == cudaSuccess) e = cudaEventRecord(hp->in[c], hp->h2d);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s, hp->in[c], 0);
+    if (e != cudaSuccess) return cuda_fail(e, "host-to-device copy");
+    st = forward_impl(q_dev, k_dev, v_dev, tau_dev, 0, 0, out_dev, lse_dev, nullptr, B, Hq, Hkv, N, D, Bq, Bk, causal,
+                      stream, nullptr, 0, g0, g1 - g0);
+    if (st != BSFA_OK) return st;
+    e = cudaEventRecord(hp->done[c], s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(hp->d2h, hp->done[c], 0);
+    if (e == cudaSuccess)
+      e = copy_cols(out_host, out_dev, rows, (size_t)Hq * D, (size_t)h0 * D, (size_t)nh * D, 2, cudaMemcpyDeviceToHost,
+                    hp->d2h);
+    if (e == cudaSuccess && lse_host)   // lse [B, Hq, N]: the chunk's heads are nh * N floats per batch entry
+      e = copy_cols(lse_host, lse_dev, (size_t)B, (size_t)Hq * N, (size_t)h0 * N, (size_t)nh * N, 4,
+                    cudaMemcpyDeviceToHost, hp->d2h);
+    if (e != cudaSuccess) return cuda_fail(e, "device-to-host copy");
+  }
+  // The caller's stream reaches the end of the call once the last result is on the host.
+  e = cudaEventRecord(hp->out, hp->d2h);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(s, hp->out, 0);
+  if (e != cudaSuccess) return cuda_fail(e, "host pipeline end");
+  return BSFA_OK;
 }
 
 bsfa_status bsfa_forward_varlen(const void* q, const void* k, const void* v, const int* cu_seqlens, int nseq,
