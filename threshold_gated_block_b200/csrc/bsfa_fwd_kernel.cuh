@@ -549,15 +549,22 @@ __device__ __forceinline__ int softmax_block(const FwdParams& p, Bars* bars, uin
   const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
   const float2 nm2 = make_float2(-m, -m);
   float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+  // In three passes (arguments, exponentials, packing and sums), which schedules
+  // the SFU and FMA work of the loop better than one fused pass.
   uint32_t pk[QC / 2];
+  float2 xv[QC / 2];
+#pragma unroll
+  for (int e = 0; e < QC / 2; ++e) xv[e] = __ffma2_rn(make_float2(sv[2 * e], sv[2 * e + 1]), sl2, nm2);
 #pragma unroll
   for (int e = 0; e < QC / 2; ++e) {
-    const float2 x = __ffma2_rn(make_float2(sv[2 * e], sv[2 * e + 1]), sl2, nm2);
-    const bool poly = (e & 3) == 3;
-    const float2 pe = poly ? exp2_poly2(x) : make_float2(ex2_approx(x.x), ex2_approx(x.y));
-    pk[e] = pack_bf16x2(pe.x, pe.y);
-    if (e & 1) acc1 = __fadd2_rn(acc1, pe);
-    else acc0 = __fadd2_rn(acc0, pe);
+    if ((e & 3) == 3) xv[e] = exp2_poly2(xv[e]);
+    else xv[e] = make_float2(ex2_approx(xv[e].x), ex2_approx(xv[e].y));
+  }
+#pragma unroll
+  for (int e = 0; e < QC / 2; ++e) {
+    pk[e] = pack_bf16x2(xv[e].x, xv[e].y);
+    if (e & 1) acc1 = __fadd2_rn(acc1, xv[e]);
+    else acc0 = __fadd2_rn(acc0, xv[e]);
   }
   if (__any_sync(0xffffffffu, !live) && !live) {   // rows this block does not update: P = 0
 #pragma unroll
