@@ -207,7 +207,7 @@ bsfa_status forward_impl(const void* q, const void* k, const void* v, const floa
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
   const int tiles = (max_seqlen + 127) / 128;
   // One persistent CTA per SM (each holds a whole SM's shared memory and TMEM);
-  // the CTAs take the units in a grid-stride loop, heaviest first.
+  // the CTAs take the units in a snake order over the heaviest-first numbering.
   const long long units = p.pair_heads ? (long long)B * (p.hq_count / 2) * tiles
                                        : (long long)B * p.hq_count * ((tiles + 1) / 2);
   const int sms = g_sm_count[dev] > 0 ? g_sm_count[dev] : 1;

@@ -52,7 +52,7 @@ struct FwdParams {
   int mask_mq, mask_mkv;   // query tiles and key blocks per sequence in the block mask
   int group;          // Hq / Hkv
   int hq_begin, hq_count;   // the query heads this launch computes (all of them unless head-sharded)
-  int units;                // work units (see decode_unit); the CTAs run them in a grid-stride loop
+  int units;                // work units (see decode_unit); each CTA runs its share (see unit_index)
   int pair_heads;     // 1: slots are query heads 2p and 2p+1 on the same rows
   int gate_gap;       // 0: the BSFA gate (block maximum against tau); 1: the gap gate, tau holding gamma
                       // (selects the kernel's GAP template argument at launch)
@@ -192,10 +192,18 @@ __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
 
 // ---------------------------------------------------------------------------- units of a persistent CTA
 
-// A CTA runs units blockIdx.x, blockIdx.x + gridDim.x, ... (units are numbered
-// heaviest first, so each CTA's share is heavy to light). Every role walks the
-// same sequence and skips the same empty units (rows past a short packed
-// sequence's end), so their barrier phases stay in step across units.
+// A CTA's k-th unit. Units are numbered heaviest first; the CTAs take them in a
+// snake order (forward through one round of gridDim.x units, backward through
+// the next), so each CTA pairs a heavier unit with a lighter one and the CTAs
+// finish together. Every role walks the same sequence and skips the same empty
+// units (rows past a short packed sequence's end), so their barrier phases stay
+// in step across units.
+__device__ __forceinline__ int unit_index(int k) {
+  const int g = gridDim.x, b = blockIdx.x;
+  const int base = (k >> 1) * 2 * g;
+  return (k & 1) ? base + 2 * g - 1 - b : base + b;
+}
+
 template <bool VARLEN>
 __device__ __forceinline__ bool unit_at(const FwdParams& p, int u, bool causal, int bk, FwdUnit& w, SeqSpan& sp) {
   w = decode_unit<VARLEN>(p, u, causal, bk, sp);
@@ -218,7 +226,7 @@ __device__ __forceinline__ void kq_producer(const FwdParams& p, const CUtensorMa
   prefetch_tensormap(tm_k);
   bool ok = true;
   int it = 0, kt = 0;               // units started, K blocks issued (over all units)
-  for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
+  for (int k = 0, u = unit_index(0); u < p.units && ok; u = unit_index(++k)) {
     FwdUnit w;
     SeqSpan sp;
     if (!unit_at<VARLEN>(p, u, CAUSAL, BK, w, sp)) continue;
@@ -286,7 +294,7 @@ __device__ __forceinline__ void v_producer(const FwdParams& p, const CUtensorMap
   prefetch_tensormap(tm_v);
   int v_count = 0, it = 0;
   bool failed = false;
-  for (int u = blockIdx.x; u < p.units && !failed; u += gridDim.x) {
+  for (int k = 0, u = unit_index(0); u < p.units && !failed; u = unit_index(++k)) {
     FwdUnit w;
     SeqSpan sp;
     if (!unit_at<VARLEN>(p, u, CAUSAL, BK, w, sp)) continue;
@@ -328,7 +336,7 @@ __device__ __forceinline__ void s_waiter(const FwdParams& p, Bars* bars) {
   volatile int* abort_flag = &bars->abort;
   const int lane = threadIdx.x & 31;
   int n0 = 0, n1 = 0;               // S tiles seen per slot (over all units): the s_full phases
-  for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
+  for (int k = 0, u = unit_index(0); u < p.units; u = unit_index(++k)) {
     FwdUnit w;
     SeqSpan sp;
     if (!unit_at<VARLEN>(p, u, CAUSAL, BK, w, sp)) continue;
@@ -383,7 +391,7 @@ __device__ __forceinline__ void mma_issuer(const FwdParams& p, uint8_t* smem, Ba
   // consumed, P tiles consumed per slot. They give every barrier's phase.
   int it = 0, kg = 0, v_count = 0, pc0 = 0, pc1 = 0;
   bool ok = true;
-  for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
+  for (int k = 0, u = unit_index(0); u < p.units && ok; u = unit_index(++k)) {
     FwdUnit w;
     SeqSpan sp;
     if (!unit_at<VARLEN>(p, u, CAUSAL, BK, w, sp)) continue;
@@ -722,7 +730,7 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, Bars* bars, uin
   int it = 0;
   uint32_t o_seen[2] = {0u, 0u};     // o_done completions per slot (over all units): the epilogue's phases
   const int sub = ((threadIdx.x >> 5) & 3) * 32 / BQ;
-  for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
+  for (int k = 0, u = unit_index(0); u < p.units; u = unit_index(++k)) {
     FwdUnit w;
     SeqSpan sp;
     if (!unit_at<VARLEN>(p, u, CAUSAL, BK, w, sp)) continue;
