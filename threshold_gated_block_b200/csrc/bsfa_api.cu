@@ -1,7 +1,6 @@
 // C ABI of the BSFA prefill forward: argument validation, TMA descriptor
 // encoding, kernel dispatch and the device status word. The declarations and
 // their contracts are in include/bsfa.h.
-#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -39,7 +38,6 @@ constexpr int kMaxDevices = 64;
 std::mutex g_dev_mutex;
 int* g_status_ptr[kMaxDevices] = {};
 int g_cc_major[kMaxDevices] = {};
-int g_sm_count[kMaxDevices] = {};
 
 bsfa_status device_setup(int dev, int** status_ptr) {
   if (dev < 0 || dev >= kMaxDevices) return fail(BSFA_ERR_UNSUPPORTED, "device index %d out of range", dev);
@@ -50,8 +48,6 @@ bsfa_status device_setup(int dev, int** status_ptr) {
     if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
     g_cc_major[dev] = major;
     if (major != 10) return fail(BSFA_ERR_UNSUPPORTED, "device %d has compute capability %d.x; sm_100 required", dev, major);
-    e = cudaDeviceGetAttribute(&g_sm_count[dev], cudaDevAttrMultiProcessorCount, dev);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute(multiprocessors)");
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_status_word);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(status word)");
@@ -206,15 +202,7 @@ bsfa_status forward_impl(const void* q, const void* k, const void* v, const floa
   p.scale = (float)(1.0 / std::sqrt((double)D));
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
   const int tiles = (max_seqlen + 127) / 128;
-  // One persistent CTA per SM (each holds a whole SM's shared memory and TMEM);
-  // the CTAs take the units in a snake order over the heaviest-first numbering.
-  const long long units = p.pair_heads ? (long long)B * (p.hq_count / 2) * tiles
-                                       : (long long)B * p.hq_count * ((tiles + 1) / 2);
-  const int sms = g_sm_count[dev] > 0 ? g_sm_count[dev] : 1;
-  const int grid = (int)std::min<long long>(units, sms);
-  if (units > 0x7fffffffLL || (units + grid - 1) / grid > 0x7fff)
-    return fail(BSFA_ERR_UNSUPPORTED, "%lld work units exceed what one launch handles", units);
-  p.units = (int)units;
+  const int grid = p.pair_heads ? B * (p.hq_count / 2) * tiles : B * p.hq_count * ((tiles + 1) / 2);
   e = (D == 64) ? bsfa::launch_fwd_d64(tq, tk, tv, p, Bq, Bk, causal != 0, block_mask != nullptr, grid, s)
                 : bsfa::launch_fwd_d128(tq, tk, tv, p, Bq, Bk, causal != 0, block_mask != nullptr, grid, s);
   if (e != cudaSuccess) return cuda_fail(e, "kernel launch");

@@ -52,7 +52,6 @@ struct FwdParams {
   int mask_mq, mask_mkv;   // query tiles and key blocks per sequence in the block mask
   int group;          // Hq / Hkv
   int hq_begin, hq_count;   // the query heads this launch computes (all of them unless head-sharded)
-  int units;                // work units (see decode_unit); each CTA runs its share (see unit_index)
   int pair_heads;     // 1: slots are query heads 2p and 2p+1 on the same rows
   int gate_gap;       // 0: the BSFA gate (block maximum against tau); 1: the gap gate, tau holding gamma
                       // (selects the kernel's GAP template argument at launch)
@@ -69,8 +68,8 @@ constexpr int kRowSplit = 2;
 constexpr int kSoftmaxWarps = 4 * kRowSplit;
 constexpr int kThreads = 32 * (kSoftmaxWarps + 4);
 constexpr int kLaunchRegs = kRowSplit == 2 ? 168 : 96;   // 65536 / kThreads, rounded down to the allocation granularity
-constexpr int kSoftmaxRegs = kRowSplit == 2 ? 208 : 104;
-constexpr int kProducerRegs = kRowSplit == 2 ? 88 : 64;
+constexpr int kSoftmaxRegs = kRowSplit == 2 ? 216 : 104;
+constexpr int kProducerRegs = kRowSplit == 2 ? 72 : 64;
 static_assert(kSoftmaxWarps * 32 * kSoftmaxRegs + 128 * kProducerRegs <= kThreads * kLaunchRegs, "register split");
 // Named barriers: 1 = the softmax warps' gate barrier; kSReadyBar + s = "S of
 // slot s is in TMEM", which the waiter warp joins once s_full says so and the
@@ -94,7 +93,7 @@ struct FwdShape {
   static constexpr uint32_t OFF_K = OFF_Q + 2 * Q_BYTES;
   static constexpr uint32_t OFF_V = OFF_K + KS * KV_BYTES;
   static constexpr uint32_t OFF_BAR = OFF_V + VS * KV_BYTES;
-  static constexpr uint32_t BAR_BYTES = 19456;                      // barriers, gate decisions, softmax exchange
+  static constexpr uint32_t BAR_BYTES = 11264;                      // barriers, gate decisions, softmax exchange
   static constexpr uint32_t SMEM_BYTES = OFF_BAR + BAR_BYTES;        // base is 1024-aligned (checked)
   static constexpr uint32_t TMEM_S0 = 0;
   static constexpr uint32_t TMEM_O0 = 2 * BK;
@@ -105,13 +104,13 @@ struct FwdShape {
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
 
-// Gate decisions of every block, one entry per (slot, block): at most this many
+// Gate decisions of every block, one bit per (slot, block): at most this many
 // key blocks per sequence.
 constexpr int kMaxKeyBlocks = 4096;
 
 template <int KS, int VS>
 struct alignas(16) FwdBarriers {
-  uint64_t q_full, q_empty;
+  uint64_t q_full;
   uint64_t k_full[KS], k_empty[KS];
   uint64_t v_full[VS], v_empty[VS];
   uint64_t s_full[2], p_full[2], o_done[2];
@@ -120,7 +119,7 @@ struct alignas(16) FwdBarriers {
   int abort;                               // any role gave up on a bounded wait
   int sm_abort[2];                         // softmax warps' agreement to stop, by block parity
   float xch[2 * kRowSplit * 128];          // partial row maxima [slot][part][row]; normalisers [part][row] at the end
-  alignas(16) uint16_t gate_dec[2][kMaxKeyBlocks];  // tag << 1 | keep (tag: the unit, see unit_tag)
+  alignas(16) uint8_t gate_dec[2][kMaxKeyBlocks];   // 0 undecided, 1 skipped, 2 kept
 };
 
 struct FwdUnit {
@@ -190,135 +189,92 @@ __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
   return mbar_wait(bar, parity, &local);
 }
 
-// ---------------------------------------------------------------------------- units of a persistent CTA
-
-// A CTA's k-th unit. Units are numbered heaviest first; the CTAs take them in a
-// snake order (forward through one round of gridDim.x units, backward through
-// the next), so each CTA pairs a heavier unit with a lighter one and the CTAs
-// finish together. Every role walks the same sequence and skips the same empty
-// units (rows past a short packed sequence's end), so their barrier phases stay
-// in step across units.
-__device__ __forceinline__ int unit_index(int k) {
-  const int g = gridDim.x, b = blockIdx.x;
-  const int base = (k >> 1) * 2 * g;
-  return (k & 1) ? base + 2 * g - 1 - b : base + b;
-}
-
-template <bool VARLEN>
-__device__ __forceinline__ bool unit_at(const FwdParams& p, int u, bool causal, int bk, FwdUnit& w, SeqSpan& sp) {
-  w = decode_unit<VARLEN>(p, u, causal, bk, sp);
-  return w.nblk[0] > 0 || w.nblk[1] > 0;
-}
-
-// Gate decisions are tagged with the unit (1 + the unit's index among this
-// CTA's units), so a decision left over from an earlier unit never reads as
-// this unit's: entry = tag << 1 | keep.
-__device__ __forceinline__ uint16_t unit_tag(int it) { return (uint16_t)((it & 0x7FFF) + 1); }
-
 // ---------------------------------------------------------------------------- K/Q producer (warp 8, one thread)
 
-template <int D, int BQ, int BK, bool CAUSAL, bool VARLEN, typename Bars>
-__device__ __forceinline__ void kq_producer(const FwdParams& p, const CUtensorMap* tm_q, const CUtensorMap* tm_k,
-                                            uint8_t* smem, Bars* bars) {
+template <int D, int BQ, int BK, bool VARLEN, typename Bars>
+__device__ __forceinline__ void kq_producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k, uint8_t* smem,
+                                            Bars* bars, const FwdUnit& w, const SeqSpan& sp) {
   using S = FwdShape<D, BQ, BK>;
   volatile int* abort_flag = &bars->abort;
   prefetch_tensormap(tm_q);
   prefetch_tensormap(tm_k);
-  bool ok = true;
-  int it = 0, kt = 0;               // units started, K blocks issued (over all units)
-  for (int k = 0, u = unit_index(0); u < p.units && ok; u = unit_index(++k)) {
-    FwdUnit w;
-    SeqSpan sp;
-    if (!unit_at<VARLEN>(p, u, CAUSAL, BK, w, sp)) continue;
-    // The Q tiles are free once every QK^T of the previous unit has completed.
-    if (!mbar_wait(&bars->q_empty, (it & 1) ^ 1, abort_flag)) { ok = false; break; }
-    const int nq = (w.nblk[0] > 0) + (w.nblk[1] > 0);
-    mbar_arrive_expect_tx(&bars->q_full, nq * S::Q_BYTES);
+  const int nq = (w.nblk[0] > 0) + (w.nblk[1] > 0);
+  mbar_arrive_expect_tx(&bars->q_full, nq * S::Q_BYTES);
 #pragma unroll
-    for (int s = 0; s < 2; ++s) {
-      if (w.nblk[s] == 0) continue;
+  for (int s = 0; s < 2; ++s) {
+    if (w.nblk[s] == 0) continue;
 #pragma unroll
-      for (int c = 0; c < S::DCH; ++c)
-        tma_load_4d(smem + S::OFF_Q + s * S::Q_BYTES + c * (S::ROWS * 128), tm_q, &bars->q_full, c * 64, w.hq[s],
-                    unit_row0<VARLEN>(sp) + w.q0[s], w.b);
-    }
-    ++it;
-    const int nblk = max(w.nblk[0], w.nblk[1]);
-    for (int t = 0; t < nblk; ++t) {
-      const int slot = kt % S::KS;
-      if (!mbar_wait(&bars->k_empty[slot], ((kt / S::KS) & 1) ^ 1, abort_flag)) { ok = false; break; }
-      mbar_arrive_expect_tx(&bars->k_full[slot], S::KV_BYTES);
+    for (int c = 0; c < S::DCH; ++c)
+      tma_load_4d(smem + S::OFF_Q + s * S::Q_BYTES + c * (S::ROWS * 128), tm_q, &bars->q_full, c * 64, w.hq[s],
+                  unit_row0<VARLEN>(sp) + w.q0[s], w.b);
+  }
+  const int nblk = max(w.nblk[0], w.nblk[1]);
+  int issued = 0;
+  for (int t = 0; t < nblk; ++t) {
+    const int slot = t % S::KS;
+    if (!mbar_wait(&bars->k_empty[slot], ((t / S::KS) & 1) ^ 1, abort_flag)) break;
+    mbar_arrive_expect_tx(&bars->k_full[slot], S::KV_BYTES);
 #pragma unroll
-      for (int c = 0; c < S::DCH; ++c)
-        tma_load_4d(smem + S::OFF_K + slot * S::KV_BYTES + c * (BK * 128), tm_k, &bars->k_full[slot], c * 64, w.kvh,
-                    unit_row0<VARLEN>(sp) + t * BK, w.b);
-      ++kt;
-    }
+    for (int c = 0; c < S::DCH; ++c)
+      tma_load_4d(smem + S::OFF_K + slot * S::KV_BYTES + c * (BK * 128), tm_k, &bars->k_full[slot], c * 64, w.kvh,
+                  unit_row0<VARLEN>(sp) + t * BK, w.b);
+    issued = t + 1;
   }
   // Copies still in flight must land before the CTA exits.
-  if (it > 0) drain_wait(&bars->q_full, (it - 1) & 1);
-  for (int t = (kt > S::KS ? kt - S::KS : 0); t < kt; ++t)
+  drain_wait(&bars->q_full, 0);
+  for (int t = (issued > S::KS ? issued - S::KS : 0); t < issued; ++t)
     drain_wait(&bars->k_full[t % S::KS], (t / S::KS) & 1);
 }
 
-// Bounded wait until slot s's gate decision for block j of the unit tagged
-// `tag` is published. The thread sleeps between looks: a tight shared-memory
-// spin would steal the bandwidth the QK^T MMAs (both operands in shared
-// memory) depend on. Returns the decision entry (tag << 1 | keep), or 0 if the
-// wait gave up.
+// Bounded wait until slot s's gate decision for block j is published. The
+// thread sleeps between looks: a tight shared-memory spin would steal the
+// bandwidth the QK^T MMAs (both operands in shared memory) depend on.
 template <typename Bars>
-__device__ __forceinline__ uint32_t wait_decided(Bars* bars, int s, int j, uint16_t tag) {
-  volatile uint16_t* dec = &bars->gate_dec[s][j];
+__device__ __forceinline__ bool wait_decided(Bars* bars, int s, int j) {
+  volatile uint8_t* dec = &bars->gate_dec[s][j];
   volatile int* abort_flag = &bars->abort;
-  uint32_t d = *dec;
-  if ((d >> 1) == tag) return d;
+  if (*dec != 0) return true;
   const uint64_t t0 = global_timer_ns();
   for (;;) {
     __nanosleep(64);
-    d = *dec;
-    if ((d >> 1) == tag) return d;
-    if (*abort_flag) return 0;
+    if (*dec != 0) return true;
+    if (*abort_flag) return false;
     if (global_timer_ns() - t0 > kWaitTimeoutNs) {
       *abort_flag = 1;
-      return 0;
+      return false;
     }
   }
 }
 
 // ---------------------------------------------------------------------------- V producer (one thread)
 
-template <int D, int BQ, int BK, bool CAUSAL, bool VARLEN, typename Bars>
-__device__ __forceinline__ void v_producer(const FwdParams& p, const CUtensorMap* tm_v, uint8_t* smem, Bars* bars) {
+template <int D, int BQ, int BK, bool VARLEN, typename Bars>
+__device__ __forceinline__ void v_producer(const CUtensorMap* tm_v, uint8_t* smem, Bars* bars, const FwdUnit& w,
+                                           const SeqSpan& sp) {
   using S = FwdShape<D, BQ, BK>;
   volatile int* abort_flag = &bars->abort;
   prefetch_tensormap(tm_v);
-  int v_count = 0, it = 0;
+  const int nblk = max(w.nblk[0], w.nblk[1]);
+  int v_count = 0;
   bool failed = false;
-  for (int k = 0, u = unit_index(0); u < p.units && !failed; u = unit_index(++k)) {
-    FwdUnit w;
-    SeqSpan sp;
-    if (!unit_at<VARLEN>(p, u, CAUSAL, BK, w, sp)) continue;
-    const uint16_t tag = unit_tag(it++);
-    const int nblk = max(w.nblk[0], w.nblk[1]);
-    for (int j = 0; j < nblk && !failed; ++j) {
-      bool loaded = false;
+  for (int j = 0; j < nblk && !failed; ++j) {
+    bool loaded = false;
 #pragma unroll
-      for (int s = 0; s < 2; ++s) {
-        if (j >= w.nblk[s]) continue;
-        const uint32_t d = wait_decided(bars, s, j, tag);
-        if (d == 0) { failed = true; break; }
-        if (!(d & 1u) || loaded) continue;     // skipped by this slot (or already requested)
-        const int slot = v_count % S::VS;
-        if (!mbar_wait(&bars->v_empty[slot], ((v_count / S::VS) & 1) ^ 1, abort_flag)) { failed = true; break; }
-        mbar_arrive_expect_tx(&bars->v_full[slot], S::KV_BYTES);
+    for (int s = 0; s < 2; ++s) {
+      if (j >= w.nblk[s]) continue;
+      if (!wait_decided(bars, s, j)) { failed = true; break; }
+      const bool keep = ((volatile uint8_t*)bars->gate_dec[s])[j] == 2;
+      if (!keep || loaded) continue;     // skipped by this slot (or already requested)
+      const int slot = v_count % S::VS;
+      if (!mbar_wait(&bars->v_empty[slot], ((v_count / S::VS) & 1) ^ 1, abort_flag)) { failed = true; break; }
+      mbar_arrive_expect_tx(&bars->v_full[slot], S::KV_BYTES);
 #pragma unroll
-        for (int c = 0; c < S::DCH; ++c)
-          tma_load_4d(smem + S::OFF_V + slot * S::KV_BYTES + c * (BK * 128), tm_v, &bars->v_full[slot], c * 64, w.kvh,
-                      unit_row0<VARLEN>(sp) + j * BK, w.b);
-        loaded = true;
-      }
-      if (loaded) ++v_count;
+      for (int c = 0; c < S::DCH; ++c)
+        tma_load_4d(smem + S::OFF_V + slot * S::KV_BYTES + c * (BK * 128), tm_v, &bars->v_full[slot], c * 64, w.kvh,
+                    unit_row0<VARLEN>(sp) + j * BK, w.b);
+      loaded = true;
     }
+    if (loaded) ++v_count;
   }
   for (int n = (v_count > S::VS ? v_count - S::VS : 0); n < v_count; ++n)
     drain_wait(&bars->v_full[n % S::VS], (n / S::VS) & 1);
@@ -331,37 +287,31 @@ __device__ __forceinline__ void v_producer(const FwdParams& p, const CUtensorMap
 // arriving, so it stays in lockstep with the softmax warps' steps even when its
 // waits give up (then it marks the block's abort flag first and joins anyway):
 // the softmax warps never wait on a barrier that cannot complete.
-template <int BK, bool CAUSAL, bool VARLEN, typename Bars>
-__device__ __forceinline__ void s_waiter(const FwdParams& p, Bars* bars) {
+template <typename Bars>
+__device__ __forceinline__ void s_waiter(Bars* bars, const FwdUnit& w) {
   volatile int* abort_flag = &bars->abort;
   const int lane = threadIdx.x & 31;
-  int n0 = 0, n1 = 0;               // S tiles seen per slot (over all units): the s_full phases
-  for (int k = 0, u = unit_index(0); u < p.units; u = unit_index(++k)) {
-    FwdUnit w;
-    SeqSpan sp;
-    if (!unit_at<VARLEN>(p, u, CAUSAL, BK, w, sp)) continue;
-    const int nblk = max(w.nblk[0], w.nblk[1]);
-    for (int j = 0; j < nblk; ++j) {
+  const int nblk = max(w.nblk[0], w.nblk[1]);
+  for (int j = 0; j < nblk; ++j) {
 #pragma unroll
-      for (int s = 0; s < 2; ++s) {
-        if (j >= w.nblk[s]) continue;
-        const int n = s ? n1++ : n0++;
-        if (lane == 0 && !mbar_wait(&bars->s_full[s], n & 1, abort_flag)) ((volatile int*)bars->sm_abort)[j & 1] = 1;
-        __syncwarp();
-        named_barrier_sync(kSReadyBar + s, kSReadyCount);
-      }
+    for (int s = 0; s < 2; ++s) {
+      if (j >= w.nblk[s]) continue;
+      if (lane == 0 && !mbar_wait(&bars->s_full[s], j & 1, abort_flag)) ((volatile int*)bars->sm_abort)[j & 1] = 1;
+      __syncwarp();
+      named_barrier_sync(kSReadyBar + s, kSReadyCount);
     }
   }
 }
 
 // ---------------------------------------------------------------------------- MMA issuer (warp 9, one thread)
 
-template <int D, int BQ, int BK, bool CAUSAL, bool VARLEN, typename Bars>
-__device__ __forceinline__ void mma_issuer(const FwdParams& p, uint8_t* smem, Bars* bars, uint32_t tmem) {
+template <int D, int BQ, int BK, typename Bars>
+__device__ __forceinline__ void mma_issuer(uint8_t* smem, Bars* bars, uint32_t tmem, const FwdUnit& w) {
   using S = FwdShape<D, BQ, BK>;
   constexpr uint32_t IDESC_QK = make_idesc_bf16(128, BK, false);   // B = K tile, K-major
   constexpr uint32_t IDESC_PV = make_idesc_bf16(128, D, true);     // B = V tile, MN-major
   volatile int* abort_flag = &bars->abort;
+  const int nblk = max(w.nblk[0], w.nblk[1]);
 
   auto qk = [&](int s, int kslot) {
     const uint32_t q_addr = smem_u32(smem + S::OFF_Q + s * S::Q_BYTES);
@@ -387,42 +337,28 @@ __device__ __forceinline__ void mma_issuer(const FwdParams& p, uint8_t* smem, Ba
     }
   };
 
-  // Counters over all of this CTA's units: units, K blocks consumed, V blocks
-  // consumed, P tiles consumed per slot. They give every barrier's phase.
-  int it = 0, kg = 0, v_count = 0, pc0 = 0, pc1 = 0;
-  bool ok = true;
-  for (int k = 0, u = unit_index(0); u < p.units && ok; u = unit_index(++k)) {
-    FwdUnit w;
-    SeqSpan sp;
-    if (!unit_at<VARLEN>(p, u, CAUSAL, BK, w, sp)) continue;
-    const int nblk = max(w.nblk[0], w.nblk[1]);
-    ok = mbar_wait(&bars->q_full, it & 1, abort_flag) &&
-         mbar_wait(&bars->k_full[kg % S::KS], (kg / S::KS) & 1, abort_flag);
-    if (!ok) break;
+  bool ok = mbar_wait(&bars->q_full, 0, abort_flag) && mbar_wait(&bars->k_full[0], 0, abort_flag);
+  if (ok) {
     tc_fence_after();
-    // QK_s(0). O of the previous unit may still be read by the epilogue: the
-    // first PV of a slot is issued only after that slot's P(0) of this unit,
-    // which the softmax warps publish after finishing the previous epilogue.
 #pragma unroll
     for (int s = 0; s < 2; ++s) {
       if (w.nblk[s] == 0) continue;
-      qk(s, kg % S::KS);
+      qk(s, 0);
       tc_commit(&bars->s_full[s]);
     }
-    tc_commit(&bars->k_empty[kg % S::KS]);
+    tc_commit(&bars->k_empty[0]);
+    int v_count = 0;
     bool pv_started[2] = {false, false};
     for (int j = 0; j < nblk && ok; ++j) {
       bool k_ready = false, v_ready = false;
       int vslot = 0;
-      const int kn = kg + j + 1;
-      const int kslot = kn % S::KS;
+      const int kslot = (j + 1) % S::KS;
 #pragma unroll
       for (int s = 0; s < 2; ++s) {
         if (j >= w.nblk[s]) continue;
-        const int n = s ? pc1++ : pc0++;
-        if (!mbar_wait(&bars->p_full[s], n & 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(&bars->p_full[s], j & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        if (((volatile uint16_t*)bars->gate_dec[s])[j] & 1u) {
+        if (((volatile uint8_t*)bars->gate_dec[s])[j] == 2) {
           if (!v_ready) {
             vslot = v_count % S::VS;
             if (!mbar_wait(&bars->v_full[vslot], (v_count / S::VS) & 1, abort_flag)) { ok = false; break; }
@@ -434,7 +370,7 @@ __device__ __forceinline__ void mma_issuer(const FwdParams& p, uint8_t* smem, Ba
         }
         if (j + 1 < w.nblk[s]) {
           if (!k_ready) {
-            if (!mbar_wait(&bars->k_full[kslot], (kn / S::KS) & 1, abort_flag)) { ok = false; break; }
+            if (!mbar_wait(&bars->k_full[kslot], ((j + 1) / S::KS) & 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
             k_ready = true;
           }
@@ -450,9 +386,6 @@ __device__ __forceinline__ void mma_issuer(const FwdParams& p, uint8_t* smem, Ba
       }
       if (k_ready) tc_commit(&bars->k_empty[kslot]);
     }
-    kg += nblk;
-    tc_commit(&bars->q_empty);             // this unit's QK^T are all issued: Q is free once they land
-    ++it;
   }
   // Every MMA issued above must complete before TMEM is released.
   tc_commit(&bars->drain);
@@ -481,7 +414,7 @@ struct SoftmaxRow {
 template <int D, int BQ, int BK, bool CAUSAL, bool WRITE_MASK, bool GAP, bool VARLEN, typename Bars>
 __device__ __forceinline__ int softmax_block(const FwdParams& p, Bars* bars, uint32_t tmem, const FwdUnit& w,
                                              const SeqSpan& sp, int s, int j, float tau, SoftmaxRow<BK>& st,
-                                             bool failed, uint16_t tag) {
+                                             bool failed) {
   using S = FwdShape<D, BQ, BK>;
   constexpr int QC = BK / kRowSplit;         // key columns per thread
   constexpr int QD = D / kRowSplit;          // output columns per thread
@@ -580,7 +513,7 @@ __device__ __forceinline__ int softmax_block(const FwdParams& p, Bars* bars, uin
     }
     // Publish the decision (one byte, no fence) so the V tile, if kept, is fetched
     // right away; the MMA warp reads it after p_full, whose arrival orders it.
-    ((volatile uint16_t*)bars->gate_dec[s])[j] = (uint16_t)((tag << 1) | (keep_any ? 1 : 0));
+    ((volatile uint8_t*)bars->gate_dec[s])[j] = keep_any ? 2 : 1;
   }
   if (!keep_any) {                 // skipped by every tile of the slot: release S, nothing else
     tc_fence_before();
@@ -670,8 +603,7 @@ __device__ __forceinline__ int softmax_block(const FwdParams& p, Bars* bars, uin
 // natural-log logsumexp over the kept set.
 template <int D, int BQ, int BK, bool VARLEN, typename Bars>
 __device__ __forceinline__ void softmax_epilogue(const FwdParams& p, Bars* bars, uint32_t tmem, const FwdUnit& w,
-                                                 const SeqSpan& sp, int s, SoftmaxRow<BK>& st, bool failed,
-                                                 uint32_t o_phase) {
+                                                 const SeqSpan& sp, int s, SoftmaxRow<BK>& st, bool failed) {
   using S = FwdShape<D, BQ, BK>;
   constexpr int QD = D / kRowSplit;
   volatile int* abort_flag = &bars->abort;
@@ -694,7 +626,7 @@ __device__ __forceinline__ void softmax_epilogue(const FwdParams& p, Bars* bars,
   const bool again = named_barrier_or(1, 32 * kSoftmaxWarps, any_failed);   // everyone has read lpart
   if (again) return;
   bool ok = true;
-  if (lane == 0) ok = mbar_wait(&bars->o_done[s], o_phase, abort_flag);
+  if (lane == 0) ok = mbar_wait(&bars->o_done[s], 0, abort_flag);
   ok = __shfl_sync(0xffffffffu, ok, 0);
   if (!ok) return;
   tc_fence_after();
@@ -725,44 +657,36 @@ __device__ __forceinline__ void softmax_epilogue(const FwdParams& p, Bars* bars,
 }
 
 template <int D, int BQ, int BK, bool CAUSAL, bool WRITE_MASK, bool GAP, bool VARLEN, typename Bars>
-__device__ __forceinline__ void softmax_role(const FwdParams& p, Bars* bars, uint32_t tmem) {
+__device__ __forceinline__ void softmax_role(const FwdParams& p, Bars* bars, uint32_t tmem, const FwdUnit& w,
+                                             const SeqSpan& sp) {
+  SoftmaxRow<BK> st;
   bool aborted = false;
-  int it = 0;
-  uint32_t o_seen[2] = {0u, 0u};     // o_done completions per slot (over all units): the epilogue's phases
+  // This thread's threshold in each slot: its query tile's column of the table
+  // (clamped to the table's last column), or the head's single value.
   const int sub = ((threadIdx.x >> 5) & 3) * 32 / BQ;
-  for (int k = 0, u = unit_index(0); u < p.units; u = unit_index(++k)) {
-    FwdUnit w;
-    SeqSpan sp;
-    if (!unit_at<VARLEN>(p, u, CAUSAL, BK, w, sp)) continue;
-    const uint16_t tag = unit_tag(it++);
-    SoftmaxRow<BK> st;
-    // This thread's threshold in each slot: its query tile's column of the table
-    // (clamped to the table's last column), or the head's single value.
-    auto tile_tau = [&](int s) {
-      const int hq = w.hq[s];
-      const int tile = w.q0[s] / BQ + sub;
-      const float t = p.tau_tiles > 0 ? p.tau[hq * p.tau_tiles + min(tile, p.tau_tiles - 1)] : p.tau[hq];
-      return GAP ? t * 1.4426950408889634f : t;   // gamma in the exp2 domain of the running maximum
-    };
-    const float tau0 = tile_tau(0), tau1 = tile_tau(1);
-    const int nblk = max(w.nblk[0], w.nblk[1]);
-    // Every step is taken even after an abort (then without work), in the
-    // waiter warp's order.
-    for (int j = 0; j < nblk; ++j) {
+  auto tile_tau = [&](int s) {
+    const int hq = w.hq[s];
+    const int tile = w.q0[s] / BQ + sub;
+    const float t = p.tau_tiles > 0 ? p.tau[hq * p.tau_tiles + min(tile, p.tau_tiles - 1)] : p.tau[hq];
+    return GAP ? t * 1.4426950408889634f : t;   // gamma in the exp2 domain of the running maximum
+  };
+  const float tau0 = tile_tau(0), tau1 = tile_tau(1);
+  const int nblk = max(w.nblk[0], w.nblk[1]);
+  // Every step is taken even after an abort (then without work), in the
+  // waiter warp's order.
+  for (int j = 0; j < nblk; ++j) {
 #pragma unroll 1
-      for (int s = 0; s < 2; ++s) {
-        if (j >= (s ? w.nblk[1] : w.nblk[0])) continue;
-        if (softmax_block<D, BQ, BK, CAUSAL, WRITE_MASK, GAP, VARLEN>(p, bars, tmem, w, sp, s, j, s ? tau1 : tau0, st,
-                                                                     aborted, tag) == 2)
-          aborted = true;
-      }
-    }
-#pragma unroll
     for (int s = 0; s < 2; ++s) {
-      if (w.nblk[s] == 0) continue;
-      softmax_epilogue<D, BQ, BK, VARLEN>(p, bars, tmem, w, sp, s, st, aborted, o_seen[s] & 1u);
-      ++o_seen[s];
+      if (j >= (s ? w.nblk[1] : w.nblk[0])) continue;
+      if (softmax_block<D, BQ, BK, CAUSAL, WRITE_MASK, GAP, VARLEN>(p, bars, tmem, w, sp, s, j, s ? tau1 : tau0, st,
+                                                                   aborted) == 2)
+        aborted = true;
     }
+  }
+#pragma unroll 1
+  for (int s = 0; s < 2; ++s) {
+    if ((s ? w.nblk[1] : w.nblk[0]) == 0) continue;
+    softmax_epilogue<D, BQ, BK, VARLEN>(p, bars, tmem, w, sp, s, st, aborted);
   }
 }
 
@@ -779,10 +703,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = smem_raw;
   Bars* bars = reinterpret_cast<Bars*>(smem + S::OFF_BAR);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  SeqSpan sp;
+  const FwdUnit w = decode_unit<VARLEN>(p, blockIdx.x, CAUSAL, BK, sp);
+  if (VARLEN && w.nblk[0] == 0 && w.nblk[1] == 0) return;   // rows past a short packed sequence's end: no work
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
-    mbar_init(&bars->q_empty, 1);
     for (int i = 0; i < S::KS; ++i) { mbar_init(&bars->k_full[i], 1); mbar_init(&bars->k_empty[i], 1); }
     for (int i = 0; i < S::VS; ++i) { mbar_init(&bars->v_full[i], 1); mbar_init(&bars->v_empty[i], 1); }
     for (int i = 0; i < 2; ++i) {
@@ -795,8 +721,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     bars->abort = 0;
     fence_mbar_init();
   }
-  // Gate decisions start with tag 0, which no unit uses; every thread clears a share.
-  for (int i = threadIdx.x; i < (int)(sizeof(bars->gate_dec) / 16); i += kThreads)
+  // Gate decisions start undecided (0); every thread clears a share.
+  for (int i = threadIdx.x; i < 2 * kMaxKeyBlocks / 16; i += kThreads)
     reinterpret_cast<uint4*>(&bars->gate_dec[0][0])[i] = make_uint4(0u, 0u, 0u, 0u);
   // The 128-byte swizzle and the descriptors assume a 1024-byte aligned base.
   if ((smem_u32(smem) & 1023u) != 0) {
@@ -814,16 +740,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < kSoftmaxWarps) {
     regs_increase<kSoftmaxRegs>();
-    softmax_role<D, BQ, BK, CAUSAL, WRITE_MASK, GAP, VARLEN>(p, bars, tmem);
+    softmax_role<D, BQ, BK, CAUSAL, WRITE_MASK, GAP, VARLEN>(p, bars, tmem, w, sp);
   } else {
     regs_decrease<kProducerRegs>();
     if (lane == 0) {
-      if (warp == kSoftmaxWarps) kq_producer<D, BQ, BK, CAUSAL, VARLEN>(p, &tm_q, &tm_k, smem, bars);
-      else if (warp == kSoftmaxWarps + 1) mma_issuer<D, BQ, BK, CAUSAL, VARLEN>(p, smem, bars, tmem);
-      else if (warp == kSoftmaxWarps + 2) v_producer<D, BQ, BK, CAUSAL, VARLEN>(p, &tm_v, smem, bars);
+      if (warp == kSoftmaxWarps) kq_producer<D, BQ, BK, VARLEN>(&tm_q, &tm_k, smem, bars, w, sp);
+      else if (warp == kSoftmaxWarps + 1) mma_issuer<D, BQ, BK>(smem, bars, tmem, w);
+      else if (warp == kSoftmaxWarps + 2) v_producer<D, BQ, BK, VARLEN>(&tm_v, smem, bars, w, sp);
     }
     __syncwarp();
-    if (warp == kSoftmaxWarps + 3) s_waiter<BK, CAUSAL, VARLEN>(p, bars);
+    if (warp == kSoftmaxWarps + 3) s_waiter(bars, w);
   }
 
   tc_fence_before();
