@@ -106,3 +106,20 @@ def test_reference_arm_prints_once_under_two_ranks():
     rec = json.loads(lines[0])
     assert rec["impl"] == "reference" and rec["n_gpus"] == 2 and rec["value"] > 0
     assert rec["e2e"]["h2d_bytes_per_step"] == 0 and rec["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_bench_flop_accounting_from_block_codes():
+    """Executed FLOPs count QK^T for every visited tile and PV for kept ones; the
+    dense-equivalent count takes both for every visited tile (a tile is 2*Bq*Bk*D)."""
+    sys.path.insert(0, ROOT)
+    import numpy as np
+    import bench
+    from threshold_gated_block_b200.inputs import CONFIGS
+    cfg = CONFIGS["c2"]
+    codes = np.array([[[[2, 3, 3], [0, 2, 3], [1, 0, 2]]]], dtype=np.uint8)   # 6 visited: 3 forced, 1 kept, 2 skipped
+    visited = int((codes != 3).sum())
+    kept = int(np.isin(codes, (1, 2)).sum())
+    tile = 2.0 * cfg.Bq * cfg.Bk * cfg.D
+    exec_f, dense_f = bench.mask_flops(codes, cfg)
+    assert exec_f == (visited + kept) * tile and dense_f == 2 * visited * tile
+    assert bench.weak_scaling_value(1e12, 4, 10.0) == 4 * 1e12 / 10e-3 / 1e12

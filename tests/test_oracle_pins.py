@@ -271,3 +271,30 @@ def test_kept_set_shrinks_as_tau_grows():
 def test_bf16_round_to_nearest_even():
     x = np.array([1.00390625, 1.01171875, -1.00390625, 1.0], dtype=np.float32)
     assert f32_to_bf16_bits(x).tolist() == [0x3F80, 0x3F82, 0xBF80, 0x3F80]
+
+
+# ----------------------------------------------------------------------------- packed mixed-length batches
+
+def test_varlen_oracle_is_each_sequence_alone():
+    """A packed batch is the per-sequence forward on each [cu[e], cu[e+1]) slice,
+    checked here against the scalar brute force of each slice; empty sequences
+    produce nothing and rows of one sequence never see another's keys."""
+    lengths = [17, 0, 40, 1, 33]
+    cfg = custom_config(N=sum(lengths), D=8, Hq=2, Hkv=1, Bq=16, Bk=16, causal=True, seed=3)
+    x = make_inputs(cfg)
+    packed = {n: x[n][0] for n in "qkv"}
+    cu = np.concatenate([[0], np.cumsum(lengths)])
+    tau = [2.0, 2.4]
+    r = O.forward_varlen(packed["q"], packed["k"], packed["v"], cu, tau, 16, 16, True)
+    assert r["out"].shape == (sum(lengths), 2, 8) and r["lse"].shape == (2, sum(lengths))
+    assert r["codes"][1] is None
+    for e, n in enumerate(lengths):
+        if n == 0:
+            continue
+        r0, r1 = int(cu[e]), int(cu[e + 1])
+        qf, kf, vf = (O.widen_bf16(packed[m][r0:r1])[None].tolist() for m in "qkv")
+        out, lse, codes = brute.brute_forward(qf, kf, vf, tau, 16, 16, True)
+        np.testing.assert_allclose(r["out"][r0:r1], np.array(out)[0], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(r["lse"][:, r0:r1], np.array(lse)[0], rtol=0, atol=1e-12)
+        for (b, hq, i, j), c in codes.items():
+            assert r["codes"][e][hq, i, j] == c
