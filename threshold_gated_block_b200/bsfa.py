@@ -215,7 +215,13 @@ def forward_varlen(q, k, v, cu_seqlens, max_seqlen: int, tau, *, Bq: int, Bk: in
         raise ValueError("cu_seqlens must be a 1-D int32 CUDA tensor")
     total, Hq, D = q.shape
     Hkv = k.shape[1]
+    if k.shape != (total, Hkv, D) or v.shape != k.shape:
+        raise ValueError("k and v must be [total, Hkv, D] with q's total and D")
+    if tau.dtype != torch.float32 or not tau.is_cuda or not tau.is_contiguous() or tau.shape != (Hq,):
+        raise ValueError("tau must be a contiguous float32 CUDA tensor with one value per query head")
     nseq = cu_seqlens.numel() - 1
+    if nseq < 1:
+        raise ValueError("cu_seqlens needs at least two offsets")
     out = torch.empty_like(q)
     lse = torch.empty((Hq, total), dtype=torch.float32, device=q.device) if want_lse else None
     mask = None
