@@ -1,4 +1,4 @@
-"""The polynomial exp2 the softmax kernel uses for half of its exponentials.
+"""The polynomial exp2 the softmax kernel uses for one in four of its exponentials.
 
 The coefficients in ptx.cuh must be the ones fit_exp2_poly.py produces, and the
 kernel's fp32 operation sequence (clamp, round via 1.5*2^23, reduce, Horner in
