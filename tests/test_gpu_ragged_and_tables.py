@@ -238,3 +238,26 @@ def test_host_buffer_call_equals_the_device_call(chunks):
     assert bsfa.bsfa_get_status(None) == bsfa.BSFA_OK
     assert np.array_equal(out.float().numpy().astype(np.float64), dev["out"])
     assert np.array_equal(lse.numpy().astype(np.float64), dev["lse"])
+
+
+# ----------------------------------------------------------------------------- the largest supported length
+
+@pytest.mark.parametrize("N,D,Bq,Bk,causal", [
+    (4096 * 64, 64, 64, 64, True),          # exactly 4096 key blocks
+    (4096 * 64 - 37, 64, 64, 64, False),    # 4096 key blocks, the last one ragged
+    (4096 * 128, 128, 128, 128, True),      # 4096 blocks of 128 keys
+])
+def test_longest_supported_sequence(N, D, Bq, Bk, causal):
+    """ceil(N/Bk) at the 4096-block limit: every per-block decision slot of a CTA
+    is used. Sampled tiles, the last two (one CTA pair) among them, with tau
+    calibrated on those tiles."""
+    cfg, x = _inputs(N, D, 1, 1, Bq, Bk, causal, seed=41)
+    mq = -(-N // Bq)
+    tiles = sorted(set(sample_tiles(cfg, 5)) | {(0, 0, mq - 2)})
+    tau = calibrate(x["q"], x["k"], Bq, Bk, causal, [0.7], tiles=tiles)[0.7]
+    gpu = run_gpu(x, tau, Bq, Bk, causal)
+    assert gpu["mask"].shape == (1, 1, mq, 4096)
+    stats = compare_tiles(x, tau, Bq, Bk, causal, gpu, tiles).check()
+    m = gpu["mask"][0, 0, mq - 1]
+    assert (m == 0).any() and (m == 1).any()
+    print(N, stats)
