@@ -119,3 +119,39 @@ def test_host_buffer_entry_rejects_bad_arguments_without_touching_cuda(lib):
     half_lse[11] = None                                                                        # lse on one side only
     assert bsfa.bsfa_forward_host(*half_lse, *shape, 2, None) == bsfa.BSFA_ERR_INVALID_ARG
     assert bsfa.bsfa_forward_host(*ptrs, 1, 8, 4, 512, 96, 128, 128, 1, 2, None) == bsfa.BSFA_ERR_UNSUPPORTED
+
+
+def test_host_buffer_binding_checks_layouts_before_any_copy():
+    """forward_host hands raw host addresses and device buffers to the C call, so
+    wrong dtypes, strides or buffer shapes must be refused before it runs."""
+    import torch
+    B, N, Hq, Hkv, D = 1, 96, 4, 2, 64
+    q = torch.zeros((B, N, Hq, D), dtype=torch.bfloat16)
+    k = torch.zeros((B, N, Hkv, D), dtype=torch.bfloat16)
+    v = torch.zeros_like(k)
+    tau = torch.zeros(Hq, dtype=torch.float32)
+    bufs = {"q": q.clone(), "k": k.clone(), "v": v.clone(), "tau": tau.clone(), "out": q.clone(),
+            "lse": torch.zeros((B, Hq, N)), "out_host": q.clone(), "lse_host": torch.zeros((B, Hq, N))}
+    bsfa._check_host_inputs(q, k, v, tau, bufs)               # consistent: accepted
+    bsfa._check_host_inputs(q, k, v, tau, None)
+
+    call = lambda *a, b=bufs: bsfa.forward_host(*a, Bq=64, Bk=64, causal=True, bufs=b)
+    bad_inputs = [
+        (q.float(), k, v, tau),                                # wrong dtype
+        (q.transpose(1, 2), k, v, tau),                        # not contiguous
+        (q, k[:, :48], v, tau),                                # k shorter than q
+        (q, k, v[..., :32].contiguous(), tau),                 # v's head dimension
+        (q, k, v, tau[:3]),                                    # one threshold short
+        (q, k, v, tau.double()),                               # wrong threshold dtype
+    ]
+    for args in bad_inputs:
+        with pytest.raises(ValueError):
+            call(*args)
+    for name, bad in (("out", torch.zeros((B, N - 1, Hq, D), dtype=torch.bfloat16)),
+                      ("k", torch.zeros((B, N, Hq, D), dtype=torch.bfloat16)),
+                      ("lse_host", torch.zeros((B, Hq, N), dtype=torch.bfloat16)),
+                      ("tau", None)):
+        b = dict(bufs)
+        b[name] = bad
+        with pytest.raises(ValueError):
+            call(q, k, v, tau, b=b)

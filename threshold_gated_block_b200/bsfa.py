@@ -246,6 +246,7 @@ def forward_host(q, k, v, tau, *, Bq: int, Bk: int, causal: bool, device=None, s
     Returns (out_host, lse_host).
     """
     import torch
+    _check_host_inputs(q, k, v, tau, bufs)
     device = torch.device("cuda") if device is None else device
     if stream is None:
         stream = torch.cuda.current_stream(device)
@@ -268,6 +269,32 @@ def forward_host(q, k, v, tau, *, Bq: int, Bk: int, causal: bool, device=None, s
         bufs["lse_host"].copy_(bufs["lse"], non_blocking=True)
     stream.synchronize()
     return bufs["out_host"], bufs["lse_host"]
+
+
+def _check_host_inputs(q, k, v, tau, bufs):
+    """The host-buffer call reads q, k, v and tau by raw address and copies into
+    ``bufs`` by size, so their layouts are checked here, before any copy."""
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.dtype != torch.bfloat16 or t.is_cuda or not t.is_contiguous() or t.dim() != 4:
+            raise ValueError(f"{name} must be a contiguous 4-D bf16 host tensor")
+    B, N, Hq, D = q.shape
+    Hkv = k.shape[2]
+    if k.shape != (B, N, Hkv, D) or v.shape != k.shape:
+        raise ValueError("k and v must be [B, N, Hkv, D] with q's B, N and D")
+    if (tau.dtype != torch.float32 or tau.is_cuda or not tau.is_contiguous() or tau.dim() not in (1, 2)
+            or tau.shape[0] != Hq):
+        raise ValueError("tau must be a contiguous float32 host tensor [Hq] or [Hq, tiles]")
+    if bufs is None:
+        return
+    want = {"q": tuple(q.shape), "k": tuple(k.shape), "v": tuple(k.shape), "tau": tuple(tau.shape),
+            "out": tuple(q.shape), "lse": (B, Hq, N), "out_host": tuple(q.shape), "lse_host": (B, Hq, N)}
+    for name, shape in want.items():
+        t = bufs.get(name)
+        if t is None or tuple(t.shape) != shape or not t.is_contiguous():
+            raise ValueError(f"bufs[{name!r}] must be a contiguous tensor of shape {shape}")
+        if t.dtype != (torch.bfloat16 if name in ("q", "k", "v", "out", "out_host") else torch.float32):
+            raise ValueError(f"bufs[{name!r}] has dtype {t.dtype}")
 
 
 def device_buffers(q_shape, kv_shape, device, tau_shape=None):
