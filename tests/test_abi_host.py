@@ -27,6 +27,19 @@ def test_header_declares_the_binding_names():
     assert _declared() == sorted(bsfa.EXPORTED)
 
 
+def test_binding_signatures_match_the_header(lib):
+    """Each ctypes declaration has the header's argument count, with a pointer
+    exactly where the header has one and an int where it has an int or enum."""
+    import ctypes
+    text = open(os.path.join(ROOT, "include", "bsfa.h")).read()
+    decls = re.findall(r"^(?:bsfa_status|const char\*)\s+(bsfa_\w+)\(([^;]*)\);", text, flags=re.M | re.S)
+    assert sorted(n for n, _ in decls) == sorted(bsfa.EXPORTED)
+    for name, args in decls:
+        params = [a.strip() for a in args.replace("\n", " ").split(",") if a.strip() not in ("", "void")]
+        want = [ctypes.c_void_p if "*" in a else ctypes.c_int for a in params]
+        assert list(getattr(lib, name).argtypes) == want, name
+
+
 def test_library_exports_every_declared_symbol(lib):
     out = subprocess.run(["nm", "-D", "--defined-only", bsfa.LIB_PATH], capture_output=True, text=True).stdout
     exported = set(re.findall(r"\bT (bsfa_\w+)", out))
