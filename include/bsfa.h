@@ -26,6 +26,15 @@
  * the same stream are ordered by the stream. The library allocates nothing per
  * call; it keeps one device status word per device (and, for bsfa_forward_host,
  * two copy streams and their events per device, created on first use).
+ *
+ * The status word is shared by every kernel the library runs on a device,
+ * whatever stream or host thread launched it: bsfa_get_status reports (and
+ * clears) a bounded-wait failure of ANY of them, not only of the caller's own
+ * stream. Callers that run forwards on several streams of one device and need
+ * to tell their failures apart must serialise their bsfa_get_status calls with
+ * their launches. Concurrent bsfa_forward_host calls on one device are
+ * serialised inside the library (each holds the device's copy pipeline from its
+ * first copy to its last).
  */
 #ifndef BSFA_H_
 #define BSFA_H_
@@ -149,7 +158,9 @@ bsfa_status bsfa_forward_heads(const void* q, const void* k, const void* v, cons
  *   chunks                             1 <= chunks <= min(Hkv, 64)
  *
  * The library creates two copy streams and their events once per device and
- * reuses them; calls on one device share them (their copies are serialised).
+ * reuses them; calls on one device share them: a call holds them (a host lock)
+ * while it enqueues, so concurrent calls from several host threads are
+ * serialised and never consume each other's events.
  * Errors as bsfa_forward; BSFA_ERR_INVALID_ARG for a bad chunk count or a
  * missing buffer.
  */
@@ -198,7 +209,9 @@ bsfa_status bsfa_validate(int B, int Hq, int Hkv, int N, int D, int Bq, int Bk, 
  * bsfa_get_status - synchronise `stream`, then read and clear the device status
  * word of the current device. Returns BSFA_ERR_DEVICE_TIMEOUT when a kernel gave
  * up on a bounded wait since the last call, BSFA_ERR_CUDA when the
- * synchronisation itself failed, else BSFA_OK.
+ * synchronisation itself failed, else BSFA_OK. The word is one per device: a
+ * failure of a kernel launched on another stream of the same device is reported
+ * here too (and cleared), even if that stream has not finished.
  */
 bsfa_status bsfa_get_status(void* stream);
 

@@ -26,8 +26,7 @@ definition directly, per query tile, with no streaming and no rescaling:
     out_r = sum_{c in C_r} exp(s_rc - m_r) v_c / l_r
     lse_r = m_r + ln l_r
 
-Readings taken where the pages are silent or garbled (each one is listed in the
-design notes):
+Readings taken where the pages are silent or garbled:
   * the score carries the 1/sqrt(d) factor of App. B.2 step (3), and tau is in
     the units of that scaled score;
   * "below the threshold" skips, so a block whose maximum equals tau is kept;

@@ -112,6 +112,23 @@ def test_varlen_entry_rejects_bad_arguments_without_touching_cuda(lib):
     assert call(16, 2, 500, D=96) == bsfa.BSFA_ERR_UNSUPPORTED      # head dimension
 
 
+def test_varlen_limit_is_per_sequence_not_per_batch(lib):
+    """The 4096-key-block limit bounds each packed sequence (max_seqlen), not the
+    packed total: a batch of many short sequences whose total exceeds 4096*Bk
+    passes the shape checks. The misaligned out pointer then stops the call
+    before any CUDA call, so the error names the alignment, not the size."""
+    total = 4096 * 64 + 4097
+    st = bsfa.bsfa_forward_varlen(16, 16, 16, 16, 300, 1000, 16, 0x1001, None, None, total, 2, 1, 64, 64, 64, 1, None)
+    assert st == bsfa.BSFA_ERR_INVALID_ARG, bsfa.bsfa_last_error()
+    assert "aligned" in bsfa.bsfa_last_error()
+    # the same total is still refused for one sequence that long
+    st = bsfa.bsfa_forward_varlen(16, 16, 16, 16, 1, total, 16, 0x1001, None, None, total, 2, 1, 64, 64, 64, 1, None)
+    assert st == bsfa.BSFA_ERR_UNSUPPORTED and "key blocks" in bsfa.bsfa_last_error()
+    # and a total whose rows overflow the 32-bit lse index
+    st = bsfa.bsfa_forward_varlen(16, 16, 16, 16, 4, 1000, 16, 16, None, None, 2**30, 4, 1, 64, 64, 64, 1, None)
+    assert st == bsfa.BSFA_ERR_UNSUPPORTED and "32-bit" in bsfa.bsfa_last_error()
+
+
 def test_head_shard_entry_rejects_bad_ranges_without_touching_cuda(lib):
     call = lambda b, c: bsfa.bsfa_forward_heads(16, 16, 16, 16, 16, None, None, 1, 8, 4, 512, 128, 128, 128, 1, b, c,
                                                 None)

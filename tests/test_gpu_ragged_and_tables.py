@@ -196,7 +196,8 @@ def test_gap_gate_on_the_8k_layer():
 @pytest.mark.parametrize("Hq,Hkv,shards", [(8, 4, 2), (8, 4, 4), (6, 6, 3)])
 def test_head_shards_equal_the_whole_layer(Hq, Hkv, shards):
     """Each shard (bsfa_forward_heads) writes exactly its heads, bit for bit what the
-    whole-layer call writes for them; other heads are left as they were."""
+    whole-layer call writes for them; other heads are left as they were. The
+    assembled shards also match the oracle on every tile."""
     cfg, x = _inputs(1000, 128, Hq, Hkv, 128, 128, True, kind="planted", seed=60 + shards)
     tau = calibrate(x["q"], x["k"], 128, 128, True, [0.5])[0.5]
     whole = run_gpu(x, tau, 128, 128, True)
@@ -219,6 +220,10 @@ def test_head_shards_equal_the_whole_layer(Hq, Hkv, shards):
         if s + 1 < shards:
             assert (o[:, :, (s + 1) * per * g:] == 7.0).all()
     assert bsfa.bsfa_get_status(None) == bsfa.BSFA_OK
+    # The shards' own output against the oracle (the mask is taken from the
+    # whole-layer call, which the bit-equality above ties to the shards).
+    sharded = {"out": o.astype(np.float64), "lse": l.astype(np.float64), "mask": whole["mask"]}
+    print(compare_tiles(x, tau, 128, 128, True, sharded, all_tiles(1, Hq, 1000, 128)).check())
 
 
 # ----------------------------------------------------------------------------- host buffers, overlapped copies
@@ -227,17 +232,22 @@ def test_head_shards_equal_the_whole_layer(Hq, Hkv, shards):
 def test_host_buffer_call_equals_the_device_call(chunks):
     """bsfa_forward_host (copies in runs of KV heads, overlapped with the kernel)
     returns exactly what the device call computes, for an uneven chunk split and a
-    ragged N."""
+    ragged N, and matches the oracle on every tile."""
     cfg, x = _inputs(900, 128, 8, 4, 128, 64, True, kind="planted", seed=70)
     tau = calibrate(x["q"], x["k"], 128, 64, True, [0.5])[0.5]
-    dev = run_gpu(x, tau, 128, 64, True, want_mask=False)
+    dev = run_gpu(x, tau, 128, 64, True, want_mask=True)
     host = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).pin_memory()
     q, k, v = (host(x[n]) for n in "qkv")
     t = torch.tensor(np.asarray(tau, dtype=np.float32)).pin_memory()
     out, lse = bsfa.forward_host(q, k, v, t, Bq=128, Bk=64, causal=True, chunks=chunks)
     assert bsfa.bsfa_get_status(None) == bsfa.BSFA_OK
-    assert np.array_equal(out.float().numpy().astype(np.float64), dev["out"])
-    assert np.array_equal(lse.numpy().astype(np.float64), dev["lse"])
+    host_res = {"out": out.float().numpy().astype(np.float64), "lse": lse.numpy().astype(np.float64),
+                "mask": dev["mask"]}
+    assert np.array_equal(host_res["out"], dev["out"])
+    assert np.array_equal(host_res["lse"], dev["lse"])
+    # The host call's own output against the oracle (the mask comes from the device
+    # call, which the bit-equality above ties to the host call's result).
+    print(compare_tiles(x, tau, 128, 64, True, host_res, all_tiles(1, 8, 900, 128)).check())
 
 
 # ----------------------------------------------------------------------------- the largest supported length

@@ -94,3 +94,32 @@ def test_varlen_equals_each_sequence_alone(Hq, Hkv):
         assert np.array_equal(l1.cpu().numpy()[0], lse[:, r0:r1]), e
         n = r1 - r0
         assert np.array_equal(m1.cpu().numpy()[0], mask[e][:, : -(-n // 128), : -(-n // 128)]), e
+
+
+def test_packed_total_beyond_the_per_sequence_block_limit():
+    """A packed batch whose total (about 283,000 rows) exceeds 4096 blocks of 64 keys,
+    made of many short sequences: the limit applies per sequence, so it runs.
+    Checked against the oracle on a seeded sample of sequences, the last among them."""
+    rng = np.random.default_rng(77)
+    lengths = [int(n) for n in rng.integers(1, 1200, size=460)]
+    total = sum(lengths)
+    assert total > 4096 * 64 and max(lengths) <= 4096 * 64
+    Hq, Hkv, D, Bq, Bk = 2, 1, 64, 64, 64
+    cfg = custom_config(B=1, N=total, D=D, Hq=Hq, Hkv=Hkv, Bq=Bq, Bk=Bk, causal=True, kind="normal", seed=78)
+    xx = make_inputs(cfg)
+    x = {n: xx[n][0] for n in "qkv"}
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    tau = calibrate(x["q"][None, :2048], x["k"][None, :2048], Bq, Bk, True, [0.5])[0.5]
+    out, lse, mask = _run_varlen(x, cu, tau, Bq, Bk, True)
+    pick = sorted(set(int(e) for e in rng.choice(len(lengths) - 1, size=12, replace=False)) | {len(lengths) - 1})
+    rep = Report()
+    for e in pick:
+        r0, r1 = int(cu[e]), int(cu[e + 1])
+        n = r1 - r0
+        xe = {name: x[name][None, r0:r1] for name in "qkv"}
+        mq, mkv = -(-n // Bq), -(-n // Bk)
+        ge = {"out": out[None, r0:r1], "lse": lse[None, :, r0:r1], "mask": mask[e][None, :, :mq, :mkv]}
+        compare_tiles(xe, tau, Bq, Bk, True, ge, all_tiles(1, Hq, n, Bq), rep)
+    stats = rep.check()
+    assert (mask == 0).any() and (mask == 1).any()
+    print(stats)

@@ -134,18 +134,23 @@ bsfa_status forward_impl(const void* q, const void* k, const void* v, const floa
                          void* out, float* lse, uint8_t* block_mask, int B, int Hq, int Hkv, int N, int D, int Bq,
                          int Bk, int causal, void* stream, const int* cu_seqlens = nullptr, int max_seqlen = 0,
                          int kv_begin = 0, int kv_count = -1) {
-  bsfa_status st = cu_seqlens ? bsfa_validate(1, Hq, Hkv, N, D, Bq, Bk, causal)
-                              : bsfa_validate(B, Hq, Hkv, N, D, Bq, Bk, causal);
-  if (st != BSFA_OK) return st;
+  bsfa_status st;
   if (cu_seqlens) {
-    if (B <= 0 || max_seqlen <= 0) return fail(BSFA_ERR_INVALID_ARG, "nseq=%d and max_seqlen=%d must be positive", B, max_seqlen);
+    // Packed sequences: the key-block limit (the per-CTA gate decisions) applies
+    // to each sequence, i.e. to max_seqlen; the packed total only has to fit the
+    // 32-bit row indices.
+    if (B <= 0 || max_seqlen <= 0 || N <= 0)
+      return fail(BSFA_ERR_INVALID_ARG, "nseq=%d, max_seqlen=%d and total=%d must be positive", B, max_seqlen, N);
+    st = bsfa_validate(1, Hq, Hkv, max_seqlen, D, Bq, Bk, causal);
+    if (st != BSFA_OK) return st;
+    if ((long long)Hq * N > 0x7fffffffLL)
+      return fail(BSFA_ERR_UNSUPPORTED, "Hq*total=%lld exceeds the 32-bit row index", (long long)Hq * N);
     if (!aligned(cu_seqlens, 4)) return fail(BSFA_ERR_INVALID_ARG, "cu_seqlens must be 4-byte aligned");
-    const long long key_blocks = ((long long)max_seqlen + Bk - 1) / Bk;
-    if (key_blocks > bsfa::kMaxKeyBlocks)
-      return fail(BSFA_ERR_UNSUPPORTED, "ceil(max_seqlen/Bk)=%lld exceeds %d key blocks", key_blocks, bsfa::kMaxKeyBlocks);
     if ((long long)B * Hq * (((long long)max_seqlen + 127) / 128) > 0x7fffffffLL)
       return fail(BSFA_ERR_UNSUPPORTED, "nseq * Hq * ceil(max_seqlen/128) exceeds the grid");
   } else {
+    st = bsfa_validate(B, Hq, Hkv, N, D, Bq, Bk, causal);
+    if (st != BSFA_OK) return st;
     max_seqlen = N;
   }
   if (kv_count < 0) kv_count = Hkv;
@@ -203,39 +208,64 @@ bsfa_status forward_impl(const void* q, const void* k, const void* v, const floa
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
   const int tiles = (max_seqlen + 127) / 128;
   const int grid = p.pair_heads ? B * (p.hq_count / 2) * tiles : B * p.hq_count * ((tiles + 1) / 2);
-  e = (D == 64) ? bsfa::launch_fwd_d64(tq, tk, tv, p, Bq, Bk, causal != 0, block_mask != nullptr, grid, s)
-                : bsfa::launch_fwd_d128(tq, tk, tv, p, Bq, Bk, causal != 0, block_mask != nullptr, grid, s);
+  e = (D == 64) ? bsfa::launch_fwd_d64(tq, tk, tv, p, Bq, Bk, causal != 0, block_mask != nullptr, grid, dev, s)
+                : bsfa::launch_fwd_d128(tq, tk, tv, p, Bq, Bk, causal != 0, block_mask != nullptr, grid, dev, s);
   if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
   return BSFA_OK;
 }
 
 // Copy streams and events of the host-buffer path, created once per device and
 // reused by every call (so a call allocates nothing). Calls on one device share
-// them, which orders (and serialises) their copies.
+// them: each call holds the device's call lock from its first record to its last
+// wait, so the events of two calls from different host threads never interleave
+// (their copies are serialised).
 constexpr int kMaxChunks = 64;
 struct HostPipe {
   cudaStream_t h2d = nullptr, d2h = nullptr;
   cudaEvent_t start = nullptr, in[kMaxChunks] = {}, done[kMaxChunks] = {}, out = nullptr;
+  std::mutex call;
 };
 HostPipe g_pipe[kMaxDevices];
 std::mutex g_pipe_mutex;
+
+void destroy_pipe_parts(HostPipe& t) {
+  if (t.h2d) cudaStreamDestroy(t.h2d);
+  if (t.d2h) cudaStreamDestroy(t.d2h);
+  if (t.start) cudaEventDestroy(t.start);
+  if (t.out) cudaEventDestroy(t.out);
+  for (int c = 0; c < kMaxChunks; ++c) {
+    if (t.in[c]) cudaEventDestroy(t.in[c]);
+    if (t.done[c]) cudaEventDestroy(t.done[c]);
+  }
+}
 
 bsfa_status host_pipe(int dev, HostPipe** pipe) {
   std::lock_guard<std::mutex> lock(g_pipe_mutex);
   HostPipe& hp = g_pipe[dev];
   if (hp.h2d == nullptr) {
-    cudaError_t e = cudaStreamCreateWithFlags(&hp.h2d, cudaStreamNonBlocking);
-    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&hp.d2h, cudaStreamNonBlocking);
-    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&hp.start, cudaEventDisableTiming);
-    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&hp.out, cudaEventDisableTiming);
+    // Created into a scratch set and published only when every part exists; on a
+    // failure the parts made so far are destroyed and the next call starts over.
+    HostPipe t;
+    cudaError_t e = cudaStreamCreateWithFlags(&t.h2d, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&t.d2h, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&t.start, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&t.out, cudaEventDisableTiming);
     for (int c = 0; c < kMaxChunks && e == cudaSuccess; ++c) {
-      e = cudaEventCreateWithFlags(&hp.in[c], cudaEventDisableTiming);
-      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&hp.done[c], cudaEventDisableTiming);
+      e = cudaEventCreateWithFlags(&t.in[c], cudaEventDisableTiming);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&t.done[c], cudaEventDisableTiming);
     }
     if (e != cudaSuccess) {
-      hp.h2d = nullptr;
+      destroy_pipe_parts(t);
       return cuda_fail(e, "creating the copy streams");
     }
+    hp.d2h = t.d2h;
+    hp.start = t.start;
+    hp.out = t.out;
+    for (int c = 0; c < kMaxChunks; ++c) {
+      hp.in[c] = t.in[c];
+      hp.done[c] = t.done[c];
+    }
+    hp.h2d = t.h2d;     // last: a non-null h2d marks the set complete
   }
   *pipe = &hp;
   return BSFA_OK;
@@ -303,6 +333,7 @@ bsfa_status bsfa_forward_host(const void* q_host, const void* k_host, const void
   HostPipe* hp = nullptr;
   st = host_pipe(dev, &hp);
   if (st != BSFA_OK) return st;
+  std::lock_guard<std::mutex> call_lock(hp->call);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int group = Hq / Hkv;
   const size_t rows = (size_t)B * N;

@@ -3,7 +3,7 @@
 
 namespace bsfa {
 cudaError_t launch_fwd_d128(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
-                            int Bq, int Bk, bool causal, bool mask, int grid, cudaStream_t s) {
-  return launch_fwd<128>(tq, tk, tv, p, Bq, Bk, causal, mask, grid, s);
+                            int Bq, int Bk, bool causal, bool mask, int grid, int dev, cudaStream_t s) {
+  return launch_fwd<128>(tq, tk, tv, p, Bq, Bk, causal, mask, grid, dev, s);
 }
 }  // namespace bsfa
