@@ -14,15 +14,17 @@
 // heads of one KV group on the same rows (GQA), or two adjacent 128-row tiles of
 // one head (MHA, odd group sizes). Each slot holds one query tile when Bq = 128,
 // two when Bq = 64. Warp roles (384 threads):
-//   warps 0-7   softmax / gate / epilogue. All eight take one slot at a time and
-//               alternate slots block by block, so one slot's softmax overlaps
-//               the other slot's MMAs. Warp w owns TMEM lanes 32*(w%4)..+31 (its
-//               rows) and one half of the key columns (w/4): two threads per row.
+//   warps 0-3   softmax / gate / epilogue of slot 0; warps 4-7 the same for
+//               slot 1. Thread r of a warpgroup owns row r of its slot (TMEM
+//               lane r) and all of its key columns, so a row maximum never
+//               leaves its thread. The two warpgroups run concurrently: while one
+//               waits on the tensor core or on its gate barrier, the other
+//               computes exponentials.
 //   warp 8      TMEM allocation + TMA loads of both Q tiles and every K block;
 //   warp 9      tcgen05.mma issue (one thread);
 //   warp 10     TMA loads of V, issued only for blocks some slot kept;
 //   warp 11     S waiter: turns each "S is in TMEM" completion into a named
-//               barrier the softmax warps start their step on.
+//               barrier the slot's warpgroup starts its step on.
 // TMEM columns: S of slot 0 and 1 ([0,Bk), [Bk,2Bk)), then O of slot 0 and 1
 // (D columns each). P is written back as bf16 over the first Bk/2 columns of its
 // slot's S and read from there as the A operand of the PV product.
@@ -63,22 +65,23 @@ struct FwdParams {
 // exp2 domain; until then P is taken against the stale maximum (values <= 2^8,
 // exact in the final O / l ratio).
 constexpr float kRescaleThreshold = 8.0f;
-// Threads that share one query row in the softmax (each holds Bk/kRowSplit key columns).
-constexpr int kRowSplit = 2;
-constexpr int kSoftmaxWarps = 4 * kRowSplit;
+// One softmax warpgroup per slot; thread r of a warpgroup owns row r of its slot.
+constexpr int kSoftmaxWarps = 8;
 constexpr int kThreads = 32 * (kSoftmaxWarps + 4);
-constexpr int kLaunchRegs = kRowSplit == 2 ? 168 : 96;   // 65536 / kThreads, rounded down to the allocation granularity
-constexpr int kSoftmaxRegs = kRowSplit == 2 ? 216 : 104;
-constexpr int kProducerRegs = kRowSplit == 2 ? 72 : 64;
+constexpr int kLaunchRegs = 168;      // 65536 / kThreads, rounded down to the allocation granularity
+constexpr int kSoftmaxRegs = 216;
+constexpr int kProducerRegs = 72;
 static_assert(kSoftmaxWarps * 32 * kSoftmaxRegs + 128 * kProducerRegs <= kThreads * kLaunchRegs, "register split");
-// Named barriers: 1 = the softmax warps' gate barrier; kSReadyBar + s = "S of
-// slot s is in TMEM", which the waiter warp joins once s_full says so and the
-// softmax warps join at the start of their step (a hardware barrier, so the
-// softmax's critical path has no shared-memory poll of the MMA's completion
-// barrier).
-constexpr uint32_t kGateBar = 1;
-constexpr uint32_t kSReadyBar = 2;
-constexpr uint32_t kSReadyCount = 32 * (kSoftmaxWarps + 1);
+// Named barriers (0 is __syncthreads):
+//   kSReadyBar + s  "S of slot s is in TMEM": the waiter warp joins once s_full
+//                   says so, the slot's warpgroup at the start of its step (a
+//                   hardware barrier, so the softmax's critical path has no
+//                   shared-memory poll of the MMA's completion barrier);
+//   kGateBar + s    the gate of slot s: an OR over its warpgroup's comparisons.
+constexpr uint32_t kSReadyBar = 1;
+constexpr uint32_t kGateBar = 3;
+constexpr uint32_t kSReadyCount = 32 * (4 + 1);
+constexpr uint32_t kGateCount = 128;
 
 template <int D, int BQ, int BK>
 struct FwdShape {
@@ -93,7 +96,7 @@ struct FwdShape {
   static constexpr uint32_t OFF_K = OFF_Q + 2 * Q_BYTES;
   static constexpr uint32_t OFF_V = OFF_K + KS * KV_BYTES;
   static constexpr uint32_t OFF_BAR = OFF_V + VS * KV_BYTES;
-  static constexpr uint32_t BAR_BYTES = 11264;                      // barriers, gate decisions, softmax exchange
+  static constexpr uint32_t BAR_BYTES = 8448;                       // barriers and gate decisions
   static constexpr uint32_t SMEM_BYTES = OFF_BAR + BAR_BYTES;        // base is 1024-aligned (checked)
   static constexpr uint32_t TMEM_S0 = 0;
   static constexpr uint32_t TMEM_O0 = 2 * BK;
@@ -117,8 +120,7 @@ struct alignas(16) FwdBarriers {
   uint64_t drain;
   uint32_t tmem_base;
   int abort;                               // any role gave up on a bounded wait
-  int sm_abort[2];                         // softmax warps' agreement to stop, by block parity
-  float xch[2 * kRowSplit * 128];          // partial row maxima [slot][part][row]; normalisers [part][row] at the end
+  int sm_abort[2][2];                      // [slot][block parity]: the waiter gave up on that step's S
   alignas(16) uint8_t gate_dec[2][kMaxKeyBlocks];   // 0 undecided, 1 skipped, 2 kept
 };
 
@@ -261,10 +263,10 @@ __device__ __forceinline__ void v_producer(const CUtensorMap* tm_v, uint8_t* sme
     bool loaded = false;
 #pragma unroll
     for (int s = 0; s < 2; ++s) {
-      if (j >= w.nblk[s]) continue;
+      if (j >= w.nblk[s] || loaded) continue;   // (once one slot keeps j, V(j) is requested)
       if (!wait_decided(bars, s, j)) { failed = true; break; }
       const bool keep = ((volatile uint8_t*)bars->gate_dec[s])[j] == 2;
-      if (!keep || loaded) continue;     // skipped by this slot (or already requested)
+      if (!keep) continue;               // skipped by this slot
       const int slot = v_count % S::VS;
       if (!mbar_wait(&bars->v_empty[slot], ((v_count / S::VS) & 1) ^ 1, abort_flag)) { failed = true; break; }
       mbar_arrive_expect_tx(&bars->v_full[slot], S::KV_BYTES);
@@ -282,10 +284,10 @@ __device__ __forceinline__ void v_producer(const CUtensorMap* tm_v, uint8_t* sme
 
 // ---------------------------------------------------------------------------- S waiter (warp 11, whole warp)
 
-// Watches s_full for every (slot, block) step in the softmax warps' order and
+// Watches s_full for every (slot, block) step in the MMA warp's issue order and
 // joins that slot's named barrier once S is in TMEM. It syncs rather than only
-// arriving, so it stays in lockstep with the softmax warps' steps even when its
-// waits give up (then it marks the block's abort flag first and joins anyway):
+// arriving, so it stays in lockstep with each warpgroup's steps even when its
+// waits give up (then it marks the step's abort flag first and joins anyway):
 // the softmax warps never wait on a barrier that cannot complete.
 template <typename Bars>
 __device__ __forceinline__ void s_waiter(Bars* bars, const FwdUnit& w) {
@@ -296,7 +298,7 @@ __device__ __forceinline__ void s_waiter(Bars* bars, const FwdUnit& w) {
 #pragma unroll
     for (int s = 0; s < 2; ++s) {
       if (j >= w.nblk[s]) continue;
-      if (lane == 0 && !mbar_wait(&bars->s_full[s], j & 1, abort_flag)) ((volatile int*)bars->sm_abort)[j & 1] = 1;
+      if (lane == 0 && !mbar_wait(&bars->s_full[s], j & 1, abort_flag)) ((volatile int*)bars->sm_abort[s])[j & 1] = 1;
       __syncwarp();
       named_barrier_sync(kSReadyBar + s, kSReadyCount);
     }
@@ -394,100 +396,79 @@ __device__ __forceinline__ void mma_issuer(uint8_t* smem, Bars* bars, uint32_t t
 
 // ---------------------------------------------------------------------------- softmax / gate / epilogue (warps 0-7)
 
-// All softmax warps work on one slot at a time and alternate between the two
-// slots block by block, so a slot's softmax always overlaps the other slot's
-// MMAs. Warp w reads TMEM lanes 32*(w%4)..+31 (its rows) and key columns
-// [(w/4)*Bk/R, (w/4+1)*Bk/R), R = kRowSplit threads sharing each row. Partial row maxima
-// cross warps through shared memory; the gate decision itself is the OR that
-// the block's named barrier computes over the threads' own comparisons.
-template <int BK>
+// Warpgroup s (warps 4s..4s+3) works on slot s alone. Thread r owns row r of the
+// slot (TMEM lane r) and every key column of it, so the row maximum is the
+// thread's own; the block maximum of a query tile is never formed: the gate
+// decision is the OR that the tile's named barrier computes over the threads'
+// own comparisons.
 struct SoftmaxRow {
-  float m[2] = {-INFINITY, -INFINITY};   // reference maximum of the exponentials per slot, exp2 domain (lazy)
-  float l[2] = {0.f, 0.f};               // this thread's share of the running normaliser per slot
-  float M[2] = {-INFINITY, -INFINITY};   // true row maximum over the kept blocks per slot, exp2 domain (gap gate)
+  float m = -INFINITY;   // reference maximum of the exponentials, exp2 domain (lazy)
+  float l = 0.f;         // running normaliser
+  float M = -INFINITY;   // true row maximum over the kept blocks, exp2 domain (gap gate)
 };
 
-// Returns 2 when the block is abandoned (a bounded wait gave up somewhere, or an
-// earlier block was abandoned: 'failed'), which every softmax thread learns
-// after the same barrier, else 0. An abandoned step still takes part in both
-// barriers, so the barrier accounting of the softmax and waiter warps agrees.
+// One step (slot s, block j). Returns false when the step is abandoned (the
+// waiter gave up on S, or an earlier step was abandoned: 'failed'); every thread
+// of the warpgroup reads the same abort flag after the same barrier, so they
+// agree. An abandoned step still takes the S-ready barrier, so the barrier
+// accounting of the warpgroup and the waiter warp agrees.
 template <int D, int BQ, int BK, bool CAUSAL, bool WRITE_MASK, bool GAP, bool VARLEN, typename Bars>
-__device__ __forceinline__ int softmax_block(const FwdParams& p, Bars* bars, uint32_t tmem, const FwdUnit& w,
-                                             const SeqSpan& sp, int s, int j, float tau, SoftmaxRow<BK>& st,
-                                             bool failed) {
+__device__ __forceinline__ bool softmax_block(const FwdParams& p, Bars* bars, uint32_t tmem, const FwdUnit& w,
+                                              const SeqSpan& sp, int s, int j, float tau, SoftmaxRow& st,
+                                              bool failed) {
   using S = FwdShape<D, BQ, BK>;
-  constexpr int QC = BK / kRowSplit;         // key columns per thread
-  constexpr int QD = D / kRowSplit;          // output columns per thread
-  volatile int* abort_flag = &bars->abort;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int c4 = warp >> 2;                  // column part
-  const int q = warp & 3;                    // TMEM lane quarter
-  const int r = q * 32 + lane;               // row within the slot, TMEM lane
+  const int lane = threadIdx.x & 31;
+  const int wq = (threadIdx.x >> 5) & 3;     // warp within the warpgroup: TMEM lane quarter
+  const int r = wq * 32 + lane;              // row within the slot, TMEM lane
   const int hq = s ? w.hq[1] : w.hq[0];
   const int q0 = s ? w.q0[1] : w.q0[0];
   const int qrow = q0 + r;
-  const int sub = r / BQ;
-  const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+  const int sub = r / BQ;                    // query tile within the slot (Bq = 64: two per slot)
+  const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
   const uint32_t s_tmem = tmem + S::TMEM_S0 + s * BK + lane_off;
-  const uint32_t o_tmem = tmem + S::TMEM_O0 + s * D + c4 * QD + lane_off;
-  // [slot][quarter][row]: one buffer per slot. Consecutive blocks alternate
-  // slots, and the other slot's barrier in between orders this block's reads
-  // before the next write to the same buffer.
-  float* rowpart = &bars->xch[s * kRowSplit * 128];
+  const uint32_t o_tmem = tmem + S::TMEM_O0 + s * D + lane_off;
+  const int len = unit_len<VARLEN>(sp, p);
 
   // S(s, j) is in TMEM once the waiter warp has arrived (it watches s_full).
-  // After an abandoned block ('failed') the step only keeps the barriers in step.
   named_barrier_sync(kSReadyBar + s, kSReadyCount);
-  const bool ok = !failed;
-  float sv[QC];
-  float pmax = -INFINITY;
-  if (ok) {
-    tc_fence_after();
-    uint32_t raw[QC];
-    if constexpr (QC == 64) tmem_ld_x64(s_tmem + c4 * QC, raw);
-    else if constexpr (QC == 32) tmem_ld_x32(s_tmem + c4 * QC, raw);
-    else tmem_ld_x16(s_tmem + c4 * QC, raw);
+  if (failed || ((volatile int*)bars->sm_abort[s])[j & 1]) return false;
+  tc_fence_after();
+  float sv[BK];
+  {
+    uint32_t raw[BK];
+    if constexpr (BK == 128) tmem_ld_x128(s_tmem, raw);
+    else tmem_ld_x64(s_tmem, raw);
 #pragma unroll
-    for (int c = 0; c < QC; ++c) sv[c] = __uint_as_float(raw[c]);
-    // Last valid key of this row: the diagonal (causal) or the sequence end. A
-    // causal padding row (qrow >= N) also sees the zero-filled keys up to qrow;
-    // it is left out of the gate and never written, and V is zero there.
-    const int k0 = j * BK + c4 * QC;
-    const int klim = CAUSAL ? qrow : unit_len<VARLEN>(sp, p) - 1;
-    if (k0 + QC - 1 > klim) {                    // this thread's columns reach past it
-#pragma unroll
-      for (int c = 0; c < QC; ++c)
-        if (k0 + c > klim) sv[c] = -INFINITY;
-    }
-    float m0 = -INFINITY, m1 = -INFINITY;
-#pragma unroll
-    for (int c = 0; c < QC; c += 4) {
-      m0 = max3(m0, sv[c], sv[c + 1]);
-      m1 = max3(m1, sv[c + 2], sv[c + 3]);
-    }
-    pmax = fmaxf(m0, m1);
+    for (int c = 0; c < BK; ++c) sv[c] = __uint_as_float(raw[c]);
   }
-  rowpart[c4 * 128 + r] = pmax;
-  // Gate: s_max * scale >= tau holds exactly when some thread's partial maximum
-  // does, so the barrier's OR over the query tile's threads is the decision.
-  // The waiter warp raises this block's abort flag before it arrives when its
-  // wait on s_full gave up, so every softmax thread reads the same value after
-  // the gate barrier.
-  // Rows past N are padding. The gap gate (tau = gamma * log2(e)) keeps the block
-  // when some row with a valid entry has no kept block yet or reaches its running
-  // maximum minus gamma.
-  const float run_max = s ? st.M[1] : st.M[0];
-  const bool above =
-      ok && qrow < unit_len<VARLEN>(sp, p) &&
-      (GAP ? (pmax > -INFINITY && (run_max == -INFINITY || pmax * p.scale_log2 >= run_max - tau))
-           : (pmax * p.scale >= tau));
-  bool any_above[S::NSUB];
-  any_above[0] = named_barrier_or(kGateBar, 32 * kSoftmaxWarps, above && (S::NSUB == 1 || sub == 0));
-  if constexpr (S::NSUB == 2) any_above[1] = named_barrier_or(kGateBar, 32 * kSoftmaxWarps, above && sub == 1);
-  if (!ok || ((volatile int*)bars->sm_abort)[j & 1]) return 2;
-  float rmax = -INFINITY;
+  // Last valid key of this row: the diagonal (causal) or the sequence end. A
+  // causal padding row (qrow >= N) also sees the zero-filled keys up to qrow;
+  // it is left out of the gate and never written, and V is zero there.
+  const int k0 = j * BK;
+  const int klim = CAUSAL ? qrow : len - 1;
+  if (k0 + BK - 1 > klim) {                    // this row's columns reach past it
 #pragma unroll
-  for (int u = 0; u < kRowSplit; ++u) rmax = fmaxf(rmax, rowpart[u * 128 + r]);
+    for (int c = 0; c < BK; ++c)
+      if (k0 + c > klim) sv[c] = -INFINITY;
+  }
+  float m0 = -INFINITY, m1 = -INFINITY;
+#pragma unroll
+  for (int c = 0; c < BK; c += 4) {
+    m0 = max3(m0, sv[c], sv[c + 1]);
+    m1 = max3(m1, sv[c + 2], sv[c + 3]);
+  }
+  const float rmax = fmaxf(m0, m1);
+  // Gate: s_max * scale >= tau holds exactly when some row's maximum does, so the
+  // barrier's OR over the query tile's threads is the decision. Rows past N are
+  // padding. The gap gate (tau = gamma * log2(e)) keeps the block when some row
+  // with a valid entry has no kept block yet or reaches its running maximum
+  // minus gamma.
+  const bool above =
+      qrow < len && (GAP ? (rmax > -INFINITY && (st.M == -INFINITY || rmax * p.scale_log2 >= st.M - tau))
+                         : (rmax * p.scale >= tau));
+  bool any_above[S::NSUB];
+  any_above[0] = named_barrier_or(kGateBar + s, kGateCount, above && (S::NSUB == 1 || sub == 0));
+  if constexpr (S::NSUB == 2) any_above[1] = named_barrier_or(kGateBar + s, kGateCount, above && sub == 1);
   int code[S::NSUB];
   bool keep_any = false;
 #pragma unroll
@@ -497,13 +478,12 @@ __device__ __forceinline__ int softmax_block(const FwdParams& p, Bars* bars, uin
     // holding a row's own key is forced even in a last tile of one row.
     const int lo = q0 + t * BQ;
     const int k_lo = j * BK;
-    const int len = unit_len<VARLEN>(sp, p);
     const bool visible = lo < len && (!CAUSAL || k_lo <= min(lo + BQ - 1, len - 1));
     const bool diag = visible && (CAUSAL ? k_lo + BK - 1 > lo : (k_lo < lo + BQ && k_lo + BK > lo));
     code[t] = !visible ? 3 : diag ? 2 : (any_above[t] ? 1 : 0);
     keep_any |= (code[t] == 1 || code[t] == 2);
   }
-  if (warp == 0 && lane == 0) {
+  if (r == 0) {
     if (WRITE_MASK) {
       const int mq = p.mask_mq, mkv = p.mask_mkv;
 #pragma unroll
@@ -519,20 +499,17 @@ __device__ __forceinline__ int softmax_block(const FwdParams& p, Bars* bars, uin
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(&bars->p_full[s]);
-    return 0;
+    return true;
   }
 
   const int my_code = (S::NSUB == 1 || sub == 0) ? code[0] : code[S::NSUB - 1];
   const bool my_keep = (my_code == 1 || my_code == 2);       // uniform within a warp
-  float m = s ? st.m[1] : st.m[0];
-  float l = s ? st.l[1] : st.l[0];
+  float m = st.m;
   bool need_rescale = false;
   float alpha = 1.f;
   if (my_keep) {
     const float mx = rmax * p.scale_log2;
-    if (GAP) {
-      if (s) st.M[1] = fmaxf(st.M[1], mx); else st.M[0] = fmaxf(st.M[0], mx);
-    }
+    if (GAP) st.M = fmaxf(st.M, mx);
     if (mx > m + kRescaleThreshold) {      // also taken on the first finite maximum
       if (m != -INFINITY) {
         alpha = ex2_approx(m - mx);
@@ -540,154 +517,123 @@ __device__ __forceinline__ int softmax_block(const FwdParams& p, Bars* bars, uin
       }
       m = mx;
     }
-    l *= alpha;
   }
   // P = 2^(s * log2(e)/sqrt(d) - m): 3 of every 4 exponentials on the SFU (ex2),
-  // 1 as a polynomial on the FMA pipe, the rest of the arithmetic in f32x2 pairs.
-  // P (bf16 pairs) goes over S columns every thread of the slot has already read.
+  // 1 as a polynomial on the FMA pipe, the rest of the arithmetic in f32x2 pairs,
+  // in three passes (arguments, exponentials, packing and sums), which schedules
+  // the SFU and FMA work better than one fused pass. P (bf16 pairs) goes over S
+  // columns this thread has already read.
   const bool live = my_keep && (m != -INFINITY);
   const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
   const float2 nm2 = make_float2(-m, -m);
   float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
-  // In three passes (arguments, exponentials, packing and sums), which schedules
-  // the SFU and FMA work of the loop better than one fused pass.
-  uint32_t pk[QC / 2];
-  float2 xv[QC / 2];
+  uint32_t pk[BK / 2];
+  float2 xv[BK / 2];
 #pragma unroll
-  for (int e = 0; e < QC / 2; ++e) xv[e] = __ffma2_rn(make_float2(sv[2 * e], sv[2 * e + 1]), sl2, nm2);
+  for (int e = 0; e < BK / 2; ++e) xv[e] = __ffma2_rn(make_float2(sv[2 * e], sv[2 * e + 1]), sl2, nm2);
 #pragma unroll
-  for (int e = 0; e < QC / 2; ++e) {
+  for (int e = 0; e < BK / 2; ++e) {
     if ((e & 3) == 3) xv[e] = exp2_poly2(xv[e]);
     else xv[e] = make_float2(ex2_approx(xv[e].x), ex2_approx(xv[e].y));
   }
 #pragma unroll
-  for (int e = 0; e < QC / 2; ++e) {
+  for (int e = 0; e < BK / 2; ++e) {
     pk[e] = pack_bf16x2(xv[e].x, xv[e].y);
     if (e & 1) acc1 = __fadd2_rn(acc1, xv[e]);
     else acc0 = __fadd2_rn(acc0, xv[e]);
   }
   if (__any_sync(0xffffffffu, !live) && !live) {   // rows this block does not update: P = 0
 #pragma unroll
-    for (int e = 0; e < QC / 2; ++e) pk[e] = 0u;
+    for (int e = 0; e < BK / 2; ++e) pk[e] = 0u;
   }
-  if (live) l += (acc0.x + acc0.y) + (acc1.x + acc1.y);
-  if constexpr (QC == 64) tmem_st_x32(s_tmem + c4 * (QC / 2), pk);
-  else if constexpr (QC == 32) tmem_st_x16(s_tmem + c4 * (QC / 2), pk);
-  else tmem_st_x8(s_tmem + c4 * (QC / 2), pk);
+  if (live) st.l = st.l * alpha + ((acc0.x + acc0.y) + (acc1.x + acc1.y));
+  if constexpr (BK == 128) tmem_st_x64(s_tmem, pk);
+  else tmem_st_x32(s_tmem, pk);
   tmem_st_wait();
 
   // O_s is quiescent here: the commit that announced S_s(j) also covered PV_s(j-1).
   if (__any_sync(0xffffffffu, need_rescale)) {
 #pragma unroll
-    for (int c = 0; c < QD / 32 + (QD < 32); ++c) {
-      constexpr int W = QD < 32 ? QD : 32;
-      uint32_t o[W];
-      if constexpr (W == 32) tmem_ld_x32(o_tmem + c * 32, o);
-      else tmem_ld_x16(o_tmem, o);
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t o[32];
+      tmem_ld_x32(o_tmem + c * 32, o);
 #pragma unroll
-      for (int e = 0; e < W; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-      if constexpr (W == 32) tmem_st_x32(o_tmem + c * 32, o);
-      else tmem_st_x16(o_tmem, o);
+      for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+      tmem_st_x32(o_tmem + c * 32, o);
     }
     tmem_st_wait();
   }
-  if (s) { st.m[1] = m; st.l[1] = l; } else { st.m[0] = m; st.l[0] = l; }
+  st.m = m;
   tc_fence_before();
   __syncwarp();
   if (lane == 0) mbar_arrive(&bars->p_full[s]);
-  return 0;
+  return true;
 }
 
-// Epilogue of one slot: the two threads of each row combine their normalisers
-// through shared memory, then each writes its D/2 output columns; lse is the
-// natural-log logsumexp over the kept set.
+// Epilogue of slot s: each thread writes its row, O / l as bf16 with 16-byte
+// stores; lse is the natural-log logsumexp over the kept set.
 template <int D, int BQ, int BK, bool VARLEN, typename Bars>
 __device__ __forceinline__ void softmax_epilogue(const FwdParams& p, Bars* bars, uint32_t tmem, const FwdUnit& w,
-                                                 const SeqSpan& sp, int s, SoftmaxRow<BK>& st, bool failed) {
+                                                 const SeqSpan& sp, int s, const SoftmaxRow& st, bool failed) {
   using S = FwdShape<D, BQ, BK>;
-  constexpr int QD = D / kRowSplit;
+  if (failed) return;                        // uniform across the warpgroup
   volatile int* abort_flag = &bars->abort;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int c4 = warp >> 2, q = warp & 3;
-  const int r = q * 32 + lane;
+  const int lane = threadIdx.x & 31;
+  const int wq = (threadIdx.x >> 5) & 3;
+  const int r = wq * 32 + lane;
   const int hq = s ? w.hq[1] : w.hq[0];
   const int q0 = s ? w.q0[1] : w.q0[0];
   const int qrow = q0 + r;
-  const float m = s ? st.m[1] : st.m[0];
-  const float l = s ? st.l[1] : st.l[0];
-  float* lpart = bars->xch;                  // [quarter][row], reused after the last block
-  // The exchange area may still be read for the last block's row maxima.
-  if (named_barrier_or(1, 32 * kSoftmaxWarps, failed || *abort_flag)) return;
-  lpart[c4 * 128 + r] = l;
-  const bool any_failed = named_barrier_or(1, 32 * kSoftmaxWarps, *abort_flag);
-  float l_row = 0.f;
-#pragma unroll
-  for (int u = 0; u < kRowSplit; ++u) l_row += lpart[u * 128 + r];
-  const bool again = named_barrier_or(1, 32 * kSoftmaxWarps, any_failed);   // everyone has read lpart
-  if (again) return;
   bool ok = true;
   if (lane == 0) ok = mbar_wait(&bars->o_done[s], 0, abort_flag);
-  ok = __shfl_sync(0xffffffffu, ok, 0);
+  ok = __shfl_sync(0xffffffffu, ok, 0);      // the TMEM loads below are warp-collective
   if (!ok) return;
   tc_fence_after();
-  const uint32_t o_tmem = tmem + S::TMEM_O0 + s * D + c4 * QD + ((uint32_t)(q * 32) << 16);
+  const uint32_t o_tmem = tmem + S::TMEM_O0 + s * D + ((uint32_t)(wq * 32) << 16);
   // Padding rows of a last tile (qrow >= N) take part in the warp's TMEM loads
   // (warp-collective) but store nothing.
   const bool row_ok = qrow < unit_len<VARLEN>(sp, p);
-  const float inv_l = 1.f / l_row;     // > 0: every row keeps its diagonal block, which holds its own key
-  uint16_t* orow = p.out + ((size_t)(w.b * p.N + unit_row0<VARLEN>(sp) + qrow) * p.Hq + hq) * D + c4 * QD;
+  const float inv_l = 1.f / st.l;     // > 0: every row keeps its diagonal block, which holds its own key
+  uint16_t* orow = p.out + ((size_t)(w.b * p.N + unit_row0<VARLEN>(sp) + qrow) * p.Hq + hq) * D;
 #pragma unroll
-  for (int c = 0; c < QD / 32 + (QD < 32); ++c) {
-    constexpr int W = QD < 32 ? QD : 32;
-    uint32_t o[W];
-    if constexpr (W == 32) tmem_ld_x32(o_tmem + c * 32, o);
-    else tmem_ld_x16(o_tmem, o);
-    uint32_t pk[W / 2];
+  for (int c = 0; c < D / 32; ++c) {
+    uint32_t o[32];
+    tmem_ld_x32(o_tmem + c * 32, o);
+    uint32_t pk[16];
 #pragma unroll
-    for (int e = 0; e < W / 2; ++e)
+    for (int e = 0; e < 16; ++e)
       pk[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
     uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
     if (row_ok) {
 #pragma unroll
-      for (int v4 = 0; v4 < W / 8; ++v4) dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+      for (int v4 = 0; v4 < 4; ++v4) dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
     }
   }
-  if (row_ok && c4 == 0 && p.lse != nullptr)
-    p.lse[(size_t)(w.b * p.Hq + hq) * p.N + unit_row0<VARLEN>(sp) + qrow] = (m + __log2f(l_row)) * 0.69314718055994531f;
+  if (row_ok && p.lse != nullptr)
+    p.lse[(size_t)(w.b * p.Hq + hq) * p.N + unit_row0<VARLEN>(sp) + qrow] = (st.m + __log2f(st.l)) * 0.69314718055994531f;
 }
 
 template <int D, int BQ, int BK, bool CAUSAL, bool WRITE_MASK, bool GAP, bool VARLEN, typename Bars>
 __device__ __forceinline__ void softmax_role(const FwdParams& p, Bars* bars, uint32_t tmem, const FwdUnit& w,
                                              const SeqSpan& sp) {
-  SoftmaxRow<BK> st;
-  bool aborted = false;
-  // This thread's threshold in each slot: its query tile's column of the table
-  // (clamped to the table's last column), or the head's single value.
+  const int s = threadIdx.x >> 7;            // this warpgroup's slot
+  const int nblk = s ? w.nblk[1] : w.nblk[0];
+  if (nblk == 0) return;                     // slot past the end of the sequence
+  // This thread's threshold: its query tile's column of the table (clamped to
+  // the table's last column), or the head's single value.
   const int sub = ((threadIdx.x >> 5) & 3) * 32 / BQ;
-  auto tile_tau = [&](int s) {
-    const int hq = w.hq[s];
-    const int tile = w.q0[s] / BQ + sub;
-    const float t = p.tau_tiles > 0 ? p.tau[hq * p.tau_tiles + min(tile, p.tau_tiles - 1)] : p.tau[hq];
-    return GAP ? t * 1.4426950408889634f : t;   // gamma in the exp2 domain of the running maximum
-  };
-  const float tau0 = tile_tau(0), tau1 = tile_tau(1);
-  const int nblk = max(w.nblk[0], w.nblk[1]);
+  const int hq = s ? w.hq[1] : w.hq[0];
+  const int tile = (s ? w.q0[1] : w.q0[0]) / BQ + sub;
+  const float t = p.tau_tiles > 0 ? p.tau[hq * p.tau_tiles + min(tile, p.tau_tiles - 1)] : p.tau[hq];
+  const float tau = GAP ? t * 1.4426950408889634f : t;   // gamma in the exp2 domain of the running maximum
+  SoftmaxRow st;
+  bool failed = false;
   // Every step is taken even after an abort (then without work), in the
   // waiter warp's order.
-  for (int j = 0; j < nblk; ++j) {
 #pragma unroll 1
-    for (int s = 0; s < 2; ++s) {
-      if (j >= (s ? w.nblk[1] : w.nblk[0])) continue;
-      if (softmax_block<D, BQ, BK, CAUSAL, WRITE_MASK, GAP, VARLEN>(p, bars, tmem, w, sp, s, j, s ? tau1 : tau0, st,
-                                                                   aborted) == 2)
-        aborted = true;
-    }
-  }
-#pragma unroll 1
-  for (int s = 0; s < 2; ++s) {
-    if ((s ? w.nblk[1] : w.nblk[0]) == 0) continue;
-    softmax_epilogue<D, BQ, BK, VARLEN>(p, bars, tmem, w, sp, s, st, aborted);
-  }
+  for (int j = 0; j < nblk; ++j)
+    failed = !softmax_block<D, BQ, BK, CAUSAL, WRITE_MASK, GAP, VARLEN>(p, bars, tmem, w, sp, s, j, tau, st, failed);
+  softmax_epilogue<D, BQ, BK, VARLEN>(p, bars, tmem, w, sp, s, st, failed);
 }
 
 // ---------------------------------------------------------------------------- kernel
@@ -713,9 +659,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < S::VS; ++i) { mbar_init(&bars->v_full[i], 1); mbar_init(&bars->v_empty[i], 1); }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars->s_full[i], 1);
-      mbar_init(&bars->p_full[i], kSoftmaxWarps);   // one arrival per softmax warp
+      mbar_init(&bars->p_full[i], 4);               // one arrival per warp of the slot's warpgroup
       mbar_init(&bars->o_done[i], 1);
-      bars->sm_abort[i] = 0;
+      bars->sm_abort[i][0] = bars->sm_abort[i][1] = 0;
     }
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
