@@ -66,15 +66,27 @@ def _stale(target: str, deps: list[str]) -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False, extra_flags: list[str] | None = None) -> str:
-    """Compile every translation unit and link libbsfa.so; returns the library path."""
-    os.makedirs(BUILD, exist_ok=True)
-    flags = NVCC_FLAGS + list(extra_flags or [])
-    headers = [os.path.join(CSRC, h) for h in HEADERS] + [os.path.join(INCLUDE, "bsfa.h")]
+TRACE_BUILD = os.path.join(PKG, "_build_trace")
+TRACE_LIB = os.path.join(PKG, "libbsfa_trace.so")
+
+
+def build(force: bool = False, verbose: bool = False, extra_flags: list[str] | None = None,
+          trace: bool = False) -> str:
+    """Compile every translation unit and link libbsfa.so; returns the library path.
+
+    trace=True builds the profiling variant instead, libbsfa_trace.so (kernels
+    compiled with BSFA_TRACE, which stamp the SM clock at fixed points of each
+    role; include/bsfa_trace.h), in its own build folder.
+    """
+    build_dir, lib = (TRACE_BUILD, TRACE_LIB) if trace else (BUILD, LIB)
+    os.makedirs(build_dir, exist_ok=True)
+    flags = NVCC_FLAGS + (["-DBSFA_TRACE"] if trace else []) + list(extra_flags or [])
+    headers = [os.path.join(CSRC, h) for h in HEADERS] + [os.path.join(INCLUDE, h)
+                                                         for h in ("bsfa.h", "bsfa_trace.h")]
     objs, jobs = [], []
     for src in SOURCES:
         s = os.path.join(CSRC, src)
-        o = os.path.join(BUILD, src.replace(".cu", ".o"))
+        o = os.path.join(build_dir, src.replace(".cu", ".o"))
         objs.append(o)
         if force or _stale(o, [s] + headers + [__file__]):
             jobs.append([nvcc(), *flags, "-c", s, "-o", o])
@@ -90,11 +102,11 @@ def build(force: bool = False, verbose: bool = False, extra_flags: list[str] | N
 
     with cf.ThreadPoolExecutor(max_workers=len(jobs) or 1) as ex:
         list(ex.map(run, jobs))
-    if jobs or _stale(LIB, objs):
+    if jobs or _stale(lib, objs):
         run([nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-Xcompiler", "-fPIC",
-             "-o", LIB, *objs])
-    return LIB
+             "-o", lib, *objs])
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv, trace="--trace" in sys.argv))

@@ -12,6 +12,9 @@
 #include <cudaTypedefs.h>
 
 #include "bsfa.h"
+#ifdef BSFA_TRACE
+#include "bsfa_trace.h"
+#endif
 #include "bsfa_launch.cuh"
 
 namespace {
@@ -86,6 +89,12 @@ bool encode_bnhd(CUtensorMap* map, const void* ptr, int B, int N, int H, int D, 
 }
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+#ifdef BSFA_TRACE
+// Trace build only: the device buffer the next launches stamp (see bsfa_trace.h).
+unsigned long long* g_trace_buf = nullptr;
+int g_trace_ctas = 0;
+#endif
 
 // One thread waits, through the same bounded wait the forward kernel uses, on an
 // mbarrier that nothing will ever arrive on. The wait gives up after its time
@@ -204,6 +213,12 @@ bsfa_status forward_impl(const void* q, const void* k, const void* v, const floa
   p.pair_heads = (p.group % 2 == 0) ? 1 : 0;
   p.hq_begin = kv_begin * p.group;
   p.hq_count = kv_count * p.group;
+  p.trace = nullptr;
+  p.trace_ctas = 0;
+#ifdef BSFA_TRACE
+  p.trace = g_trace_buf;
+  p.trace_ctas = g_trace_ctas;
+#endif
   p.scale = (float)(1.0 / std::sqrt((double)D));
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
   const int tiles = (max_seqlen + 127) / 128;
@@ -430,5 +445,17 @@ const char* bsfa_status_string(bsfa_status s) {
 }
 
 const char* bsfa_last_error(void) { return g_last_error; }
+
+#ifdef BSFA_TRACE
+bsfa_status bsfa_trace_attach(void* buf, int ctas) {
+  if (ctas < 0 || (ctas > 0 && buf == nullptr) || !aligned(buf, 8))
+    return fail(BSFA_ERR_INVALID_ARG, "trace buffer %p for %d CTAs", buf, ctas);
+  g_trace_buf = static_cast<unsigned long long*>(buf);
+  g_trace_ctas = ctas;
+  return BSFA_OK;
+}
+
+int bsfa_trace_stride(void) { return bsfa::kTraceStride; }
+#endif
 
 }  // extern "C"

@@ -21,10 +21,13 @@
 //               waits on the tensor core or on its gate barrier, the other
 //               computes exponentials.
 //   warp 8      TMEM allocation + TMA loads of both Q tiles and every K block;
-//   warp 9      tcgen05.mma issue (one thread);
+//   warp 9      tcgen05.mma issue (one thread), both slots in a fixed order, each
+//               step released by a named barrier the slot's warpgroup arrives on
+//               once its P is stored;
 //   warp 10     TMA loads of V, issued only for blocks some slot kept;
-//   warp 11     S waiter: turns each "S is in TMEM" completion into a named
-//               barrier the slot's warpgroup starts its step on.
+//   warp 11     S waiter: all 32 lanes poll each "S is in TMEM" completion and
+//               turn it into a named barrier the slot's warpgroup starts its
+//               step on.
 // TMEM columns: S of slot 0 and 1 ([0,Bk), [Bk,2Bk)), then O of slot 0 and 1
 // (D columns each). P is written back as bf16 over the first Bk/2 columns of its
 // slot's S and read from there as the A operand of the PV product.
@@ -59,7 +62,50 @@ struct FwdParams {
                       // (selects the kernel's GAP template argument at launch)
   float scale;        // 1/sqrt(D): the gate compares s_max(raw) * scale against tau
   float scale_log2;   // log2(e)/sqrt(D): exponent scale of the softmax
+  // Cycle trace of the first trace_ctas CTAs (kernels built with BSFA_TRACE only;
+  // null otherwise): kTraceStride SM-clock stamps per CTA, laid out as below.
+  unsigned long long* trace;
+  int trace_ctas;
 };
+
+// Trace layout per CTA (clock64 stamps; steps past kTraceSteps are not recorded):
+//   [0] start, [1] SM id, [2] end, [3 + w] warp w's clock right after the first
+//   __syncthreads (the clocks of an SM's sub-partitions need not agree: these
+//   give each warp's offset)
+//   softmax  kTrSoftmax + (s * kTraceSteps + j) * 8 + e, by the slot's row-0 thread:
+//            e = 0 S-ready barrier passed, 1 TMEM fence done, 2 scores loaded, 3 row
+//            maxima taken, 4 gate barrier passed, 5 exponentials done, 6 P stored,
+//            7 P-ready arrival
+//   mma      kTrMma + (s * kTraceSteps + j) * 4 + e: 0 P-ready passed, 1 V ready (kept
+//            blocks), 2 PV issued, 3 next QK issued and committed
+//   waiter   kTrWait + s * kTraceSteps + j: s_full seen
+//   V        kTrV + j * 2 + e: 0 decision seen, 1 load issued (or found not needed)
+//   K        kTrK + j: load issued
+//   epilogue kTrEpi + s * 2 + e: 0 o_done seen, 1 rows written
+constexpr int kTraceSteps = 64;
+constexpr int kTrSoftmax = 16;
+constexpr int kTrMma = kTrSoftmax + 2 * kTraceSteps * 8;
+constexpr int kTrWait = kTrMma + 2 * kTraceSteps * 4;
+constexpr int kTrV = kTrWait + 2 * kTraceSteps;
+constexpr int kTrK = kTrV + 2 * kTraceSteps;
+constexpr int kTrEpi = kTrK + kTraceSteps;
+constexpr int kTraceStride = 1920;
+static_assert(kTrEpi + 4 <= kTraceStride, "trace layout");
+
+#ifdef BSFA_TRACE
+__device__ __forceinline__ void trace_at(const FwdParams& p, int idx) {
+  if (p.trace != nullptr && (int)blockIdx.x < p.trace_ctas)
+    p.trace[(size_t)blockIdx.x * kTraceStride + idx] = clock64();
+}
+__device__ __forceinline__ void trace_step(const FwdParams& p, int base, int j, int e, int per) {
+  if (j < kTraceSteps) trace_at(p, base + j * per + e);
+}
+#define BSFA_TRACE_AT(p, idx) trace_at((p), (idx))
+#define BSFA_TRACE_STEP(p, base, j, e, per) trace_step((p), (base), (j), (e), (per))
+#else
+#define BSFA_TRACE_AT(p, idx) ((void)0)
+#define BSFA_TRACE_STEP(p, base, j, e, per) ((void)0)
+#endif
 
 // O is rescaled only when the running maximum grows by more than 2^8 in the
 // exp2 domain; until then P is taken against the stale maximum (values <= 2^8,
@@ -77,11 +123,19 @@ static_assert(kSoftmaxWarps * 32 * kSoftmaxRegs + 128 * kProducerRegs <= kThread
 //                   says so, the slot's warpgroup at the start of its step (a
 //                   hardware barrier, so the softmax's critical path has no
 //                   shared-memory poll of the MMA's completion barrier);
-//   kGateBar + s    the gate of slot s: an OR over its warpgroup's comparisons.
+//   kGateBar + s    the gate of slot s: an OR over its warpgroup's comparisons;
+//   kPReadyBar + s  P of slot s is stored (or the block was skipped, or the step
+//                   abandoned): the warpgroup arrives, the whole MMA warp syncs.
 constexpr uint32_t kSReadyBar = 1;
 constexpr uint32_t kGateBar = 3;
+constexpr uint32_t kPReadyBar = 5;
 constexpr uint32_t kSReadyCount = 32 * (4 + 1);
 constexpr uint32_t kGateCount = 128;
+constexpr uint32_t kPReadyCount = 32 * (4 + 1);
+
+__device__ __forceinline__ void named_barrier_arrive(uint32_t id, uint32_t count) {
+  asm volatile("barrier.cta.arrive.aligned %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
 
 template <int D, int BQ, int BK>
 struct FwdShape {
@@ -116,7 +170,7 @@ struct alignas(16) FwdBarriers {
   uint64_t q_full;
   uint64_t k_full[KS], k_empty[KS];
   uint64_t v_full[VS], v_empty[VS];
-  uint64_t s_full[2], p_full[2], o_done[2];
+  uint64_t s_full[2], o_done[2];
   uint64_t drain;
   uint32_t tmem_base;
   int abort;                               // any role gave up on a bounded wait
@@ -194,8 +248,8 @@ __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
 // ---------------------------------------------------------------------------- K/Q producer (warp 8, one thread)
 
 template <int D, int BQ, int BK, bool VARLEN, typename Bars>
-__device__ __forceinline__ void kq_producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k, uint8_t* smem,
-                                            Bars* bars, const FwdUnit& w, const SeqSpan& sp) {
+__device__ __forceinline__ void kq_producer(const FwdParams& p, const CUtensorMap* tm_q, const CUtensorMap* tm_k,
+                                            uint8_t* smem, Bars* bars, const FwdUnit& w, const SeqSpan& sp) {
   using S = FwdShape<D, BQ, BK>;
   volatile int* abort_flag = &bars->abort;
   prefetch_tensormap(tm_q);
@@ -220,6 +274,7 @@ __device__ __forceinline__ void kq_producer(const CUtensorMap* tm_q, const CUten
     for (int c = 0; c < S::DCH; ++c)
       tma_load_4d(smem + S::OFF_K + slot * S::KV_BYTES + c * (BK * 128), tm_k, &bars->k_full[slot], c * 64, w.kvh,
                   unit_row0<VARLEN>(sp) + t * BK, w.b);
+    BSFA_TRACE_STEP(p, kTrK, t, 0, 1);
     issued = t + 1;
   }
   // Copies still in flight must land before the CTA exits.
@@ -251,8 +306,8 @@ __device__ __forceinline__ bool wait_decided(Bars* bars, int s, int j) {
 // ---------------------------------------------------------------------------- V producer (one thread)
 
 template <int D, int BQ, int BK, bool VARLEN, typename Bars>
-__device__ __forceinline__ void v_producer(const CUtensorMap* tm_v, uint8_t* smem, Bars* bars, const FwdUnit& w,
-                                           const SeqSpan& sp) {
+__device__ __forceinline__ void v_producer(const FwdParams& p, const CUtensorMap* tm_v, uint8_t* smem, Bars* bars,
+                                           const FwdUnit& w, const SeqSpan& sp) {
   using S = FwdShape<D, BQ, BK>;
   volatile int* abort_flag = &bars->abort;
   prefetch_tensormap(tm_v);
@@ -265,6 +320,7 @@ __device__ __forceinline__ void v_producer(const CUtensorMap* tm_v, uint8_t* sme
     for (int s = 0; s < 2; ++s) {
       if (j >= w.nblk[s] || loaded) continue;   // (once one slot keeps j, V(j) is requested)
       if (!wait_decided(bars, s, j)) { failed = true; break; }
+      BSFA_TRACE_STEP(p, kTrV, j, 0, 2);
       const bool keep = ((volatile uint8_t*)bars->gate_dec[s])[j] == 2;
       if (!keep) continue;               // skipped by this slot
       const int slot = v_count % S::VS;
@@ -276,6 +332,7 @@ __device__ __forceinline__ void v_producer(const CUtensorMap* tm_v, uint8_t* sme
                     unit_row0<VARLEN>(sp) + j * BK, w.b);
       loaded = true;
     }
+    BSFA_TRACE_STEP(p, kTrV, j, 1, 2);
     if (loaded) ++v_count;
   }
   for (int n = (v_count > S::VS ? v_count - S::VS : 0); n < v_count; ++n)
@@ -285,12 +342,14 @@ __device__ __forceinline__ void v_producer(const CUtensorMap* tm_v, uint8_t* sme
 // ---------------------------------------------------------------------------- S waiter (warp 11, whole warp)
 
 // Watches s_full for every (slot, block) step in the MMA warp's issue order and
-// joins that slot's named barrier once S is in TMEM. It syncs rather than only
+// joins that slot's named barrier once S is in TMEM. All 32 lanes poll, so the
+// warp is converged when it reaches the (warp-aligned) barrier and none of its
+// lanes can arrive before the poll has seen S. It syncs rather than only
 // arriving, so it stays in lockstep with each warpgroup's steps even when its
 // waits give up (then it marks the step's abort flag first and joins anyway):
 // the softmax warps never wait on a barrier that cannot complete.
 template <typename Bars>
-__device__ __forceinline__ void s_waiter(Bars* bars, const FwdUnit& w) {
+__device__ __forceinline__ void s_waiter(const FwdParams& p, Bars* bars, const FwdUnit& w) {
   volatile int* abort_flag = &bars->abort;
   const int lane = threadIdx.x & 31;
   const int nblk = max(w.nblk[0], w.nblk[1]);
@@ -298,7 +357,9 @@ __device__ __forceinline__ void s_waiter(Bars* bars, const FwdUnit& w) {
 #pragma unroll
     for (int s = 0; s < 2; ++s) {
       if (j >= w.nblk[s]) continue;
-      if (lane == 0 && !mbar_wait(&bars->s_full[s], j & 1, abort_flag)) ((volatile int*)bars->sm_abort[s])[j & 1] = 1;
+      const bool got = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[s], j & 1, abort_flag));
+      if (!got && lane == 0) ((volatile int*)bars->sm_abort[s])[j & 1] = 1;
+      if (lane == 0) BSFA_TRACE_STEP(p, kTrWait + s * kTraceSteps, j, 0, 1);
       __syncwarp();
       named_barrier_sync(kSReadyBar + s, kSReadyCount);
     }
@@ -308,7 +369,8 @@ __device__ __forceinline__ void s_waiter(Bars* bars, const FwdUnit& w) {
 // ---------------------------------------------------------------------------- MMA issuer (warp 9, one thread)
 
 template <int D, int BQ, int BK, typename Bars>
-__device__ __forceinline__ void mma_issuer(uint8_t* smem, Bars* bars, uint32_t tmem, const FwdUnit& w) {
+__device__ __forceinline__ void mma_issuer(const FwdParams& p, uint8_t* smem, Bars* bars, uint32_t tmem,
+                                           const FwdUnit& w) {
   using S = FwdShape<D, BQ, BK>;
   constexpr uint32_t IDESC_QK = make_idesc_bf16(128, BK, false);   // B = K tile, K-major
   constexpr uint32_t IDESC_PV = make_idesc_bf16(128, D, true);     // B = V tile, MN-major
@@ -339,8 +401,11 @@ __device__ __forceinline__ void mma_issuer(uint8_t* smem, Bars* bars, uint32_t t
     }
   };
 
-  bool ok = mbar_wait(&bars->q_full, 0, abort_flag) && mbar_wait(&bars->k_full[0], 0, abort_flag);
-  if (ok) {
+  const bool leader = (threadIdx.x & 31) == 0;
+  bool ok = true;
+  if (leader) ok = mbar_wait(&bars->q_full, 0, abort_flag) && mbar_wait(&bars->k_full[0], 0, abort_flag);
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  if (ok && leader) {
     tc_fence_after();
 #pragma unroll
     for (int s = 0; s < 2; ++s) {
@@ -349,49 +414,69 @@ __device__ __forceinline__ void mma_issuer(uint8_t* smem, Bars* bars, uint32_t t
       tc_commit(&bars->s_full[s]);
     }
     tc_commit(&bars->k_empty[0]);
-    int v_count = 0;
-    bool pv_started[2] = {false, false};
-    for (int j = 0; j < nblk && ok; ++j) {
-      bool k_ready = false, v_ready = false;
-      int vslot = 0;
-      const int kslot = (j + 1) % S::KS;
+  }
+  int v_count = 0;
+  bool pv_started[2] = {false, false};
+  // The whole warp syncs on every (slot, block) step's P-ready barrier with the
+  // slot's warpgroup, even after a give-up; lane 0 issues.
+  for (int j = 0; j < nblk; ++j) {
+    bool k_ready = false, v_ready = false;
+    int vslot = 0;
+    const int kslot = (j + 1) % S::KS;
 #pragma unroll
-      for (int s = 0; s < 2; ++s) {
-        if (j >= w.nblk[s]) continue;
-        if (!mbar_wait(&bars->p_full[s], j & 1, abort_flag)) { ok = false; break; }
+    for (int s = 0; s < 2; ++s) {
+      if (j >= w.nblk[s]) continue;
+      __syncwarp();                           // the barrier is warp-aligned: lane 0 may still be issuing
+      named_barrier_sync(kPReadyBar + s, kPReadyCount);
+      if (leader && ok) {
+        BSFA_TRACE_STEP(p, kTrMma + s * kTraceSteps * 4, j, 0, 4);
         tc_fence_after();
-        if (((volatile uint8_t*)bars->gate_dec[s])[j] == 2) {
+        if (*abort_flag) ok = false;
+        if (ok && ((volatile uint8_t*)bars->gate_dec[s])[j] == 2) {
           if (!v_ready) {
             vslot = v_count % S::VS;
-            if (!mbar_wait(&bars->v_full[vslot], (v_count / S::VS) & 1, abort_flag)) { ok = false; break; }
-            tc_fence_after();
-            v_ready = true;
+            if (!mbar_wait(&bars->v_full[vslot], (v_count / S::VS) & 1, abort_flag)) ok = false;
+            else { tc_fence_after(); v_ready = true; }
           }
-          pv(s, vslot, !pv_started[s]);
-          pv_started[s] = true;
+          if (ok) {
+            BSFA_TRACE_STEP(p, kTrMma + s * kTraceSteps * 4, j, 1, 4);
+            pv(s, vslot, !pv_started[s]);
+            pv_started[s] = true;
+            BSFA_TRACE_STEP(p, kTrMma + s * kTraceSteps * 4, j, 2, 4);
+          }
         }
-        if (j + 1 < w.nblk[s]) {
-          if (!k_ready) {
-            if (!mbar_wait(&bars->k_full[kslot], ((j + 1) / S::KS) & 1, abort_flag)) { ok = false; break; }
-            tc_fence_after();
-            k_ready = true;
+        if (ok) {
+          if (j + 1 < w.nblk[s]) {
+            if (!k_ready) {
+              if (!mbar_wait(&bars->k_full[kslot], ((j + 1) / S::KS) & 1, abort_flag)) ok = false;
+              else { tc_fence_after(); k_ready = true; }
+            }
+            if (ok) {
+              qk(s, kslot);
+              tc_commit(&bars->s_full[s]);
+            }
+          } else {
+            tc_commit(&bars->o_done[s]);
           }
-          qk(s, kslot);
-          tc_commit(&bars->s_full[s]);
-        } else {
-          tc_commit(&bars->o_done[s]);     // this slot's last block: O is final once this lands
+          BSFA_TRACE_STEP(p, kTrMma + s * kTraceSteps * 4, j, 3, 4);
         }
       }
+    }
+    if (leader) {
       if (v_ready) {
         tc_commit(&bars->v_empty[vslot]);
         ++v_count;
       }
       if (k_ready) tc_commit(&bars->k_empty[kslot]);
     }
+    __syncwarp();
   }
   // Every MMA issued above must complete before TMEM is released.
-  tc_commit(&bars->drain);
-  drain_wait(&bars->drain, 0);
+  if (leader) {
+    tc_commit(&bars->drain);
+    drain_wait(&bars->drain, 0);
+  }
+  __syncwarp();
 }
 
 // ---------------------------------------------------------------------------- softmax / gate / epilogue (warps 0-7)
@@ -431,8 +516,15 @@ __device__ __forceinline__ bool softmax_block(const FwdParams& p, Bars* bars, ui
 
   // S(s, j) is in TMEM once the waiter warp has arrived (it watches s_full).
   named_barrier_sync(kSReadyBar + s, kSReadyCount);
-  if (failed || ((volatile int*)bars->sm_abort[s])[j & 1]) return false;
+  const int tr = kTrSoftmax + s * kTraceSteps * 8;
+  (void)tr;
+  if (r == 0) BSFA_TRACE_STEP(p, tr, j, 0, 8);
+  if (failed || ((volatile int*)bars->sm_abort[s])[j & 1]) {
+    named_barrier_arrive(kPReadyBar + s, kPReadyCount);    // the MMA warp takes every step's barrier too
+    return false;
+  }
   tc_fence_after();
+  if (r == 0) BSFA_TRACE_STEP(p, tr, j, 1, 8);
   float sv[BK];
   {
     uint32_t raw[BK];
@@ -441,6 +533,7 @@ __device__ __forceinline__ bool softmax_block(const FwdParams& p, Bars* bars, ui
 #pragma unroll
     for (int c = 0; c < BK; ++c) sv[c] = __uint_as_float(raw[c]);
   }
+  if (r == 0) BSFA_TRACE_STEP(p, tr, j, 2, 8);
   // Last valid key of this row: the diagonal (causal) or the sequence end. A
   // causal padding row (qrow >= N) also sees the zero-filled keys up to qrow;
   // it is left out of the gate and never written, and V is zero there.
@@ -451,13 +544,16 @@ __device__ __forceinline__ bool softmax_block(const FwdParams& p, Bars* bars, ui
     for (int c = 0; c < BK; ++c)
       if (k0 + c > klim) sv[c] = -INFINITY;
   }
-  float m0 = -INFINITY, m1 = -INFINITY;
+  float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
 #pragma unroll
-  for (int c = 0; c < BK; c += 4) {
+  for (int c = 0; c < BK; c += 8) {
     m0 = max3(m0, sv[c], sv[c + 1]);
     m1 = max3(m1, sv[c + 2], sv[c + 3]);
+    m2 = max3(m2, sv[c + 4], sv[c + 5]);
+    m3 = max3(m3, sv[c + 6], sv[c + 7]);
   }
-  const float rmax = fmaxf(m0, m1);
+  const float rmax = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+  if (r == 0) BSFA_TRACE_STEP(p, tr, j, 3, 8);
   // Gate: s_max * scale >= tau holds exactly when some row's maximum does, so the
   // barrier's OR over the query tile's threads is the decision. Rows past N are
   // padding. The gap gate (tau = gamma * log2(e)) keeps the block when some row
@@ -469,6 +565,7 @@ __device__ __forceinline__ bool softmax_block(const FwdParams& p, Bars* bars, ui
   bool any_above[S::NSUB];
   any_above[0] = named_barrier_or(kGateBar + s, kGateCount, above && (S::NSUB == 1 || sub == 0));
   if constexpr (S::NSUB == 2) any_above[1] = named_barrier_or(kGateBar + s, kGateCount, above && sub == 1);
+  if (r == 0) BSFA_TRACE_STEP(p, tr, j, 4, 8);
   int code[S::NSUB];
   bool keep_any = false;
 #pragma unroll
@@ -492,13 +589,14 @@ __device__ __forceinline__ bool softmax_block(const FwdParams& p, Bars* bars, ui
           p.mask[((size_t)(unit_seq<VARLEN>(w, sp) * p.Hq + hq) * mq + (q0 / BQ + t)) * mkv + j] = (uint8_t)code[t];
     }
     // Publish the decision (one byte, no fence) so the V tile, if kept, is fetched
-    // right away; the MMA warp reads it after p_full, whose arrival orders it.
+    // right away; the MMA warp reads it after the P-ready barrier, which orders it.
     ((volatile uint8_t*)bars->gate_dec[s])[j] = keep_any ? 2 : 1;
   }
   if (!keep_any) {                 // skipped by every tile of the slot: release S, nothing else
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) mbar_arrive(&bars->p_full[s]);
+    named_barrier_arrive(kPReadyBar + s, kPReadyCount);
+    if (r == 0) BSFA_TRACE_STEP(p, tr, j, 7, 8);
     return true;
   }
 
@@ -547,9 +645,11 @@ __device__ __forceinline__ bool softmax_block(const FwdParams& p, Bars* bars, ui
     for (int e = 0; e < BK / 2; ++e) pk[e] = 0u;
   }
   if (live) st.l = st.l * alpha + ((acc0.x + acc0.y) + (acc1.x + acc1.y));
+  if (r == 0) BSFA_TRACE_STEP(p, tr, j, 5, 8);
   if constexpr (BK == 128) tmem_st_x64(s_tmem, pk);
   else tmem_st_x32(s_tmem, pk);
   tmem_st_wait();
+  if (r == 0) BSFA_TRACE_STEP(p, tr, j, 6, 8);
 
   // O_s is quiescent here: the commit that announced S_s(j) also covered PV_s(j-1).
   if (__any_sync(0xffffffffu, need_rescale)) {
@@ -566,7 +666,8 @@ __device__ __forceinline__ bool softmax_block(const FwdParams& p, Bars* bars, ui
   st.m = m;
   tc_fence_before();
   __syncwarp();
-  if (lane == 0) mbar_arrive(&bars->p_full[s]);
+  named_barrier_arrive(kPReadyBar + s, kPReadyCount);
+  if (r == 0) BSFA_TRACE_STEP(p, tr, j, 7, 8);
   return true;
 }
 
@@ -588,6 +689,7 @@ __device__ __forceinline__ void softmax_epilogue(const FwdParams& p, Bars* bars,
   if (lane == 0) ok = mbar_wait(&bars->o_done[s], 0, abort_flag);
   ok = __shfl_sync(0xffffffffu, ok, 0);      // the TMEM loads below are warp-collective
   if (!ok) return;
+  if (r == 0) BSFA_TRACE_AT(p, kTrEpi + s * 2);
   tc_fence_after();
   const uint32_t o_tmem = tmem + S::TMEM_O0 + s * D + ((uint32_t)(wq * 32) << 16);
   // Padding rows of a last tile (qrow >= N) take part in the warp's TMEM loads
@@ -611,6 +713,7 @@ __device__ __forceinline__ void softmax_epilogue(const FwdParams& p, Bars* bars,
   }
   if (row_ok && p.lse != nullptr)
     p.lse[(size_t)(w.b * p.Hq + hq) * p.N + unit_row0<VARLEN>(sp) + qrow] = (st.m + __log2f(st.l)) * 0.69314718055994531f;
+  if (r == 0) BSFA_TRACE_AT(p, kTrEpi + s * 2 + 1);
 }
 
 template <int D, int BQ, int BK, bool CAUSAL, bool WRITE_MASK, bool GAP, bool VARLEN, typename Bars>
@@ -654,12 +757,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (VARLEN && w.nblk[0] == 0 && w.nblk[1] == 0) return;   // rows past a short packed sequence's end: no work
 
   if (threadIdx.x == 0) {
+#ifdef BSFA_TRACE
+    BSFA_TRACE_AT(p, 0);
+    if (p.trace != nullptr && (int)blockIdx.x < p.trace_ctas) {
+      unsigned smid;
+      asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+      p.trace[(size_t)blockIdx.x * kTraceStride + 1] = smid;
+    }
+#endif
     mbar_init(&bars->q_full, 1);
     for (int i = 0; i < S::KS; ++i) { mbar_init(&bars->k_full[i], 1); mbar_init(&bars->k_empty[i], 1); }
     for (int i = 0; i < S::VS; ++i) { mbar_init(&bars->v_full[i], 1); mbar_init(&bars->v_empty[i], 1); }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars->s_full[i], 1);
-      mbar_init(&bars->p_full[i], 4);               // one arrival per warp of the slot's warpgroup
       mbar_init(&bars->o_done[i], 1);
       bars->sm_abort[i][0] = bars->sm_abort[i][1] = 0;
     }
@@ -681,6 +791,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
   }
   __syncthreads();
+  if (lane == 0) BSFA_TRACE_AT(p, 3 + warp);
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 
@@ -690,12 +801,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     regs_decrease<kProducerRegs>();
     if (lane == 0) {
-      if (warp == kSoftmaxWarps) kq_producer<D, BQ, BK, VARLEN>(&tm_q, &tm_k, smem, bars, w, sp);
-      else if (warp == kSoftmaxWarps + 1) mma_issuer<D, BQ, BK>(smem, bars, tmem, w);
-      else if (warp == kSoftmaxWarps + 2) v_producer<D, BQ, BK, VARLEN>(&tm_v, smem, bars, w, sp);
+      if (warp == kSoftmaxWarps) kq_producer<D, BQ, BK, VARLEN>(p, &tm_q, &tm_k, smem, bars, w, sp);
+      else if (warp == kSoftmaxWarps + 2) v_producer<D, BQ, BK, VARLEN>(p, &tm_v, smem, bars, w, sp);
     }
     __syncwarp();
-    if (warp == kSoftmaxWarps + 3) s_waiter(bars, w);
+    if (warp == kSoftmaxWarps + 1) mma_issuer<D, BQ, BK>(p, smem, bars, tmem, w);
+    if (warp == kSoftmaxWarps + 3) s_waiter(p, bars, w);
   }
 
   tc_fence_before();
@@ -705,6 +816,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_dealloc(tmem, S::TMEM_COLS);
   }
   if (threadIdx.x == 0 && ((volatile int*)&bars->abort)[0]) atomicOr(p.status, 1);
+  if (threadIdx.x == 0) BSFA_TRACE_AT(p, 2);
 }
 
 }  // namespace bsfa
