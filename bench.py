@@ -62,6 +62,10 @@ def parse():
                     help="gate with the stored per-position (fixed-k) table level that keeps K blocks per tile")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU-oracle baseline")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="leave out the skip sweep (the default c2 line also times the 32K layer at 30/50/70/90%% "
+                         "skip and dense, one GPU)")
+    ap.add_argument("--sweep-config", default="c3", help="workload of the skip sweep")
     ap.add_argument("--gate", choices=["tau", "gap"], default="tau",
                     help="tau: the BSFA gate; gap: the gap-to-running-maximum gate, for comparison")
     ap.add_argument("--gamma", type=float, default=-1.0, help="gamma of the gap gate (scaled-score units)")
@@ -275,6 +279,73 @@ def run_reference(args):
     return 0
 
 
+# ----------------------------------------------------------------------------- skip sweep (extra keys of the line)
+
+def skip_sweep(cfg_name, dev, steps, warmup, flush, peak):
+    """Time one layer of ``cfg_name`` at every stored per-head skip level and at
+    tau = -inf (the dense comparator), with L2 flushed between launches: the
+    evidence that wall time falls with the skip fraction. One JSON object."""
+    import torch
+    from threshold_gated_block_b200 import bsfa
+    cfg = CONFIGS[cfg_name]
+    with open(TAUS) as f:
+        levels = json.load(f)[cfg.name]["taus"]
+    x = make_inputs(cfg)
+    to_dev = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+    q, k, v = to_dev(x["q"]), to_dev(x["k"]), to_dev(x["v"])
+    del x
+    out = torch.empty_like(q)
+    lse = torch.empty((cfg.B, cfg.Hq, cfg.N), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def run(t):
+        st = bsfa.bsfa_forward(q, k, v, t, out, lse, None, cfg.B, cfg.Hq, cfg.Hkv, cfg.N, cfg.D, cfg.Bq, cfg.Bk,
+                               cfg.causal, stream)
+        if st != bsfa.BSFA_OK:
+            raise RuntimeError(bsfa.bsfa_last_error())
+
+    def timed_ms(t):
+        for _ in range(warmup):
+            run(t)
+        ev = []
+        for _ in range(steps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            run(t)
+            b.record(stream)
+            ev.append((a, b))
+        torch.cuda.synchronize(dev)
+        return sum(a.elapsed_time(b) for a, b in ev) / steps
+
+    sampler = ClockSampler(dev.index or 0, None)
+    time.sleep(0.2)
+    dense = torch.full((cfg.Hq,), float("-inf"), dtype=torch.float32, device=dev)
+    dense_ms = timed_ms(dense)
+    points = []
+    for p_s, taus in sorted(levels.items(), key=lambda kv: float(kv[0])):
+        t = torch.tensor(taus, dtype=torch.float32, device=dev)
+        _, _, mask = bsfa.forward(q, k, v, t, Bq=cfg.Bq, Bk=cfg.Bk, causal=cfg.causal, want_lse=False,
+                                  want_mask=True)
+        m = mask.cpu().numpy()
+        del mask
+        exec_f, dense_f = mask_flops(m, cfg)
+        ms = timed_ms(t)
+        gated = np.isin(m, (0, 1))
+        points.append({"target_skip": float(p_s), "achieved_skip": float((m == 0).sum() / max(gated.sum(), 1)),
+                       "ms": ms, "speedup_vs_dense": dense_ms / ms,
+                       "exec_tflops": exec_f / (ms * 1e-3) / 1e12, "dense_equiv_tflops": dense_f / (ms * 1e-3) / 1e12,
+                       "frac": exec_f / (ms * 1e-3) / 1e12 / peak})
+    clocks = sampler.stop()
+    if bsfa.bsfa_get_status(stream) != bsfa.BSFA_OK:
+        raise RuntimeError(f"device status: {bsfa.bsfa_last_error()}")
+    del q, k, v, out, lse
+    torch.cuda.empty_cache()
+    ms_list = [pt["ms"] for pt in points]
+    return {"workload": f"{cfg.name}: {cfg.description}", "steps": steps, "warmup": warmup, "dense_ms": dense_ms,
+            "points": points, "monotone": all(a > b for a, b in zip(ms_list, ms_list[1:])), "clocks": clocks}
+
+
 # ----------------------------------------------------------------------------- our arm
 
 def run_ours(args):
@@ -417,6 +488,10 @@ def run_ours(args):
         if peaks.get("bf16_tflops"):
             peak, peak_src = float(peaks["bf16_tflops"]), "measured (MEASURED_PEAKS.json bf16_tflops, burst)"
     traffic = measured_traffic(cfg, p)
+    sweep = None
+    if world == 1 and not args.no_sweep and not heads and args.config == "c2" and args.gate == "tau" \
+            and args.tau_table is None:
+        sweep = skip_sweep(args.sweep_config, dev, max(3, min(args.steps, 10)), 3, flush, peak)
 
     line = None
     if rank == 0:
@@ -440,6 +515,8 @@ def run_ours(args):
         }
         if e2e is not None:
             line["e2e"] = e2e
+        if sweep is not None:
+            line["skip_sweep"] = sweep
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

@@ -216,6 +216,23 @@ bsfa_status bsfa_validate(int B, int Hq, int Hkv, int N, int D, int Bq, int Bk, 
 bsfa_status bsfa_get_status(void* stream);
 
 /*
+ * bsfa_get_debug_counts - synchronise `stream`, then read and clear the debug
+ * counters of the current device: the V tiles loaded and the PV products issued
+ * by every launch that wrote a block mask (block_mask != NULL) since the last
+ * call. Launches without a block mask count nothing and carry no counting code.
+ * They show the skip of §4.3 / §4.4 directly: a CTA loads the V tile of block j
+ * once if some of its query tiles kept j, and issues one PV product per (128-row
+ * slot, kept block). Like the status word, the counters are one pair per device,
+ * shared by all streams and host threads.
+ *
+ *   v_tiles, pv_products   host pointers, written (must be non-null)
+ *
+ * Returns BSFA_ERR_INVALID_ARG for a null pointer, BSFA_ERR_CUDA if the
+ * synchronisation or a copy fails, else BSFA_OK.
+ */
+bsfa_status bsfa_get_debug_counts(void* stream, unsigned long long* v_tiles, unsigned long long* pv_products);
+
+/*
  * bsfa_selftest_lost_arrival - exercise the failure path on the device: one
  * thread waits, through the forward kernel's bounded wait, on a barrier that
  * nothing arrives on (the shape of a lost arrival). After the wait's time limit

@@ -11,7 +11,7 @@ def _synthetic(nblk=6, skew=0):
     """A trace whose waiter and MMA warps read clocks `skew` cycles ahead of warp 0."""
     tr = np.zeros(2048, dtype=np.int64)
     for w in range(12):
-        tr[3 + w] = 500 + (skew if w in (T.mma_warp(0), T.mma_warp(1)) else 0)
+        tr[3 + w] = 500 + (skew if w in (T.MMA_WARP, T.WAIT_WARP) else 0)
     t = 1000
     for j in range(nblk):
         for s in range(2):

@@ -8,7 +8,7 @@ loudly.
 The functions named like the C entry points (``bsfa_forward``,
 ``bsfa_forward_tau_table``, ``bsfa_forward_gap``, ``bsfa_forward_heads``, ``bsfa_forward_host``,
 ``bsfa_forward_varlen``, ``bsfa_validate``,
-``bsfa_get_status``,
+``bsfa_get_status``, ``bsfa_get_debug_counts``,
 ``bsfa_selftest_lost_arrival``, ``bsfa_status_string``, ``bsfa_last_error``)
 take the same arguments; pointer arguments accept an int
 address, None, or a torch tensor (its ``data_ptr()``). ``forward`` and
@@ -29,8 +29,8 @@ BSFA_ERR_CUDA = 3
 BSFA_ERR_DEVICE_TIMEOUT = 4
 
 EXPORTED = ("bsfa_forward", "bsfa_forward_tau_table", "bsfa_forward_gap", "bsfa_forward_heads", "bsfa_forward_host",
-            "bsfa_forward_varlen", "bsfa_validate", "bsfa_get_status", "bsfa_selftest_lost_arrival",
-            "bsfa_status_string", "bsfa_last_error")
+            "bsfa_forward_varlen", "bsfa_validate", "bsfa_get_status", "bsfa_get_debug_counts",
+            "bsfa_selftest_lost_arrival", "bsfa_status_string", "bsfa_last_error")
 
 _lib = None
 
@@ -66,6 +66,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.bsfa_validate.restype = i
     lib.bsfa_get_status.argtypes = [vp]
     lib.bsfa_get_status.restype = i
+    lib.bsfa_get_debug_counts.argtypes = [vp, vp, vp]
+    lib.bsfa_get_debug_counts.restype = i
     lib.bsfa_selftest_lost_arrival.argtypes = [vp]
     lib.bsfa_selftest_lost_arrival.restype = i
     lib.bsfa_status_string.argtypes = [i]
@@ -138,6 +140,19 @@ def bsfa_validate(B, Hq, Hkv, N, D, Bq, Bk, causal) -> int:
 
 def bsfa_get_status(stream=None) -> int:
     return load().bsfa_get_status(_stream(stream))
+
+
+def bsfa_get_debug_counts(stream, v_tiles, pv_products) -> int:
+    """v_tiles, pv_products: ctypes.c_ulonglong objects (passed by reference) or int addresses."""
+    conv = lambda x: ctypes.addressof(x) if isinstance(x, ctypes.c_ulonglong) else _ptr(x)
+    return load().bsfa_get_debug_counts(_stream(stream), conv(v_tiles), conv(pv_products))
+
+
+def debug_counts(stream=None) -> tuple[int, int]:
+    """(V tiles loaded, PV products issued) by mask-writing launches since the last read; clears them."""
+    v, pv = ctypes.c_ulonglong(0), ctypes.c_ulonglong(0)
+    _check(bsfa_get_debug_counts(stream, v, pv))
+    return v.value, pv.value
 
 
 def bsfa_selftest_lost_arrival(stream=None) -> int:

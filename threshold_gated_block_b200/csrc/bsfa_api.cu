@@ -36,13 +36,16 @@ bsfa_status cuda_fail(cudaError_t e, const char* what) {
 // One status word per device: kernels OR a nonzero value into it when they give
 // up on a bounded wait.
 __device__ int g_status_word;
+// Per device: V tiles loaded and PV products issued by mask-writing launches.
+__device__ unsigned long long g_debug_counts[2];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_dev_mutex;
 int* g_status_ptr[kMaxDevices] = {};
+unsigned long long* g_counts_ptr[kMaxDevices] = {};
 int g_cc_major[kMaxDevices] = {};
 
-bsfa_status device_setup(int dev, int** status_ptr) {
+bsfa_status device_setup(int dev, int** status_ptr, unsigned long long** counts_ptr = nullptr) {
   if (dev < 0 || dev >= kMaxDevices) return fail(BSFA_ERR_UNSUPPORTED, "device index %d out of range", dev);
   std::lock_guard<std::mutex> lock(g_dev_mutex);
   if (g_status_ptr[dev] == nullptr) {
@@ -54,10 +57,15 @@ bsfa_status device_setup(int dev, int** status_ptr) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_status_word);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(status word)");
+    void* c = nullptr;
+    e = cudaGetSymbolAddress(&c, g_debug_counts);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(debug counters)");
+    g_counts_ptr[dev] = static_cast<unsigned long long*>(c);
     g_status_ptr[dev] = static_cast<int*>(p);
   }
   if (g_cc_major[dev] != 10) return fail(BSFA_ERR_UNSUPPORTED, "device %d is not sm_100", dev);
   *status_ptr = g_status_ptr[dev];
+  if (counts_ptr) *counts_ptr = g_counts_ptr[dev];
   return BSFA_OK;
 }
 
@@ -175,7 +183,8 @@ bsfa_status forward_impl(const void* q, const void* k, const void* v, const floa
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   int* status_ptr = nullptr;
-  st = device_setup(dev, &status_ptr);
+  unsigned long long* counts_ptr = nullptr;
+  st = device_setup(dev, &status_ptr, &counts_ptr);
   if (st != BSFA_OK) return st;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -203,6 +212,7 @@ bsfa_status forward_impl(const void* q, const void* k, const void* v, const floa
   p.lse = lse;
   p.mask = block_mask;
   p.status = status_ptr;
+  p.counts = counts_ptr;
   p.B = B;
   p.Hq = Hq;
   p.Hkv = Hkv;
@@ -417,6 +427,28 @@ bsfa_status bsfa_get_status(void* stream) {
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(clear status word)");
     return fail(BSFA_ERR_DEVICE_TIMEOUT, "a kernel gave up on a bounded wait (status word 0x%x)", word);
   }
+  return BSFA_OK;
+}
+
+bsfa_status bsfa_get_debug_counts(void* stream, unsigned long long* v_tiles, unsigned long long* pv_products) {
+  if (!v_tiles || !pv_products) return fail(BSFA_ERR_INVALID_ARG, "v_tiles and pv_products must be non-null");
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  int dev = 0;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  int* status_ptr = nullptr;
+  unsigned long long* counts_ptr = nullptr;
+  bsfa_status st = device_setup(dev, &status_ptr, &counts_ptr);
+  if (st != BSFA_OK) return st;
+  unsigned long long h[2] = {0, 0};
+  e = cudaMemcpy(h, counts_ptr, sizeof(h), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(debug counters)");
+  const unsigned long long zero[2] = {0, 0};
+  e = cudaMemcpy(counts_ptr, zero, sizeof(zero), cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(clear debug counters)");
+  *v_tiles = h[0];
+  *pv_products = h[1];
   return BSFA_OK;
 }
 

@@ -48,6 +48,9 @@ struct FwdParams {
   float* lse;         // [B, Hq, N] or null
   uint8_t* mask;      // [B, Hq, N/Bq, N/Bk] or null
   int* status;        // device status word
+  // Mask-writing (debug) launches only: [0] V tiles loaded, [1] PV products issued
+  // (one per slot and kept block), accumulated over launches.
+  unsigned long long* counts;
   int B, Hq, Hkv, N;  // N need not be a multiple of the tile sizes: rows and keys >= N are masked
   // Packed variable-length batch (the kernel's VARLEN variants; null otherwise):
   // sequence e holds rows [cu_seqlens[e], cu_seqlens[e+1]) of the N = total rows,
@@ -305,7 +308,7 @@ __device__ __forceinline__ bool wait_decided(Bars* bars, int s, int j) {
 
 // ---------------------------------------------------------------------------- V producer (one thread)
 
-template <int D, int BQ, int BK, bool VARLEN, typename Bars>
+template <int D, int BQ, int BK, bool VARLEN, bool COUNT, typename Bars>
 __device__ __forceinline__ void v_producer(const FwdParams& p, const CUtensorMap* tm_v, uint8_t* smem, Bars* bars,
                                            const FwdUnit& w, const SeqSpan& sp) {
   using S = FwdShape<D, BQ, BK>;
@@ -331,6 +334,7 @@ __device__ __forceinline__ void v_producer(const FwdParams& p, const CUtensorMap
         tma_load_4d(smem + S::OFF_V + slot * S::KV_BYTES + c * (BK * 128), tm_v, &bars->v_full[slot], c * 64, w.kvh,
                     unit_row0<VARLEN>(sp) + j * BK, w.b);
       loaded = true;
+      if (COUNT) atomicAdd(&p.counts[0], 1ull);
     }
     BSFA_TRACE_STEP(p, kTrV, j, 1, 2);
     if (loaded) ++v_count;
@@ -368,7 +372,7 @@ __device__ __forceinline__ void s_waiter(const FwdParams& p, Bars* bars, const F
 
 // ---------------------------------------------------------------------------- MMA issuer (warp 9, one thread)
 
-template <int D, int BQ, int BK, typename Bars>
+template <int D, int BQ, int BK, bool COUNT, typename Bars>
 __device__ __forceinline__ void mma_issuer(const FwdParams& p, uint8_t* smem, Bars* bars, uint32_t tmem,
                                            const FwdUnit& w) {
   using S = FwdShape<D, BQ, BK>;
@@ -442,6 +446,7 @@ __device__ __forceinline__ void mma_issuer(const FwdParams& p, uint8_t* smem, Ba
             BSFA_TRACE_STEP(p, kTrMma + s * kTraceSteps * 4, j, 1, 4);
             pv(s, vslot, !pv_started[s]);
             pv_started[s] = true;
+            if (COUNT) atomicAdd(&p.counts[1], 1ull);
             BSFA_TRACE_STEP(p, kTrMma + s * kTraceSteps * 4, j, 2, 4);
           }
         }
@@ -518,6 +523,7 @@ __device__ __forceinline__ bool softmax_block(const FwdParams& p, Bars* bars, ui
   named_barrier_sync(kSReadyBar + s, kSReadyCount);
   const int tr = kTrSoftmax + s * kTraceSteps * 8;
   (void)tr;
+  const bool trace_me = r == 0;
   if (r == 0) BSFA_TRACE_STEP(p, tr, j, 0, 8);
   if (failed || ((volatile int*)bars->sm_abort[s])[j & 1]) {
     named_barrier_arrive(kPReadyBar + s, kPReadyCount);    // the MMA warp takes every step's barrier too
@@ -625,29 +631,30 @@ __device__ __forceinline__ bool softmax_block(const FwdParams& p, Bars* bars, ui
   const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
   const float2 nm2 = make_float2(-m, -m);
   float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
-  uint32_t pk[BK / 2];
-  float2 xv[BK / 2];
+  const bool zero_p = __any_sync(0xffffffffu, !live) && !live;   // rows this block does not update: P = 0
+  constexpr int H = BK / 4;                  // pairs per half
 #pragma unroll
-  for (int e = 0; e < BK / 2; ++e) xv[e] = __ffma2_rn(make_float2(sv[2 * e], sv[2 * e + 1]), sl2, nm2);
+  for (int h = 0; h < 2; ++h) {
+    uint32_t pk[H];
+    float2 xv[H];
 #pragma unroll
-  for (int e = 0; e < BK / 2; ++e) {
-    if ((e & 3) == 3) xv[e] = exp2_poly2(xv[e]);
-    else xv[e] = make_float2(ex2_approx(xv[e].x), ex2_approx(xv[e].y));
-  }
+    for (int e = 0; e < H; ++e) xv[e] = __ffma2_rn(make_float2(sv[2 * (h * H + e)], sv[2 * (h * H + e) + 1]), sl2, nm2);
 #pragma unroll
-  for (int e = 0; e < BK / 2; ++e) {
-    pk[e] = pack_bf16x2(xv[e].x, xv[e].y);
-    if (e & 1) acc1 = __fadd2_rn(acc1, xv[e]);
-    else acc0 = __fadd2_rn(acc0, xv[e]);
-  }
-  if (__any_sync(0xffffffffu, !live) && !live) {   // rows this block does not update: P = 0
+    for (int e = 0; e < H; ++e) {
+      if ((e & 3) == 3) xv[e] = exp2_poly2(xv[e]);
+      else xv[e] = make_float2(ex2_approx(xv[e].x), ex2_approx(xv[e].y));
+    }
 #pragma unroll
-    for (int e = 0; e < BK / 2; ++e) pk[e] = 0u;
+    for (int e = 0; e < H; ++e) {
+      pk[e] = zero_p ? 0u : pack_bf16x2(xv[e].x, xv[e].y);
+      if (e & 1) acc1 = __fadd2_rn(acc1, xv[e]);
+      else acc0 = __fadd2_rn(acc0, xv[e]);
+    }
+    if constexpr (H == 32) tmem_st_x32(s_tmem + h * H, pk);
+    else tmem_st_x16(s_tmem + h * H, pk);
   }
   if (live) st.l = st.l * alpha + ((acc0.x + acc0.y) + (acc1.x + acc1.y));
-  if (r == 0) BSFA_TRACE_STEP(p, tr, j, 5, 8);
-  if constexpr (BK == 128) tmem_st_x64(s_tmem, pk);
-  else tmem_st_x32(s_tmem, pk);
+  if (trace_me) BSFA_TRACE_STEP(p, tr, j, 5, 8);
   tmem_st_wait();
   if (r == 0) BSFA_TRACE_STEP(p, tr, j, 6, 8);
 
@@ -802,10 +809,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     regs_decrease<kProducerRegs>();
     if (lane == 0) {
       if (warp == kSoftmaxWarps) kq_producer<D, BQ, BK, VARLEN>(p, &tm_q, &tm_k, smem, bars, w, sp);
-      else if (warp == kSoftmaxWarps + 2) v_producer<D, BQ, BK, VARLEN>(p, &tm_v, smem, bars, w, sp);
+      else if (warp == kSoftmaxWarps + 2) v_producer<D, BQ, BK, VARLEN, WRITE_MASK>(p, &tm_v, smem, bars, w, sp);
     }
     __syncwarp();
-    if (warp == kSoftmaxWarps + 1) mma_issuer<D, BQ, BK>(p, smem, bars, tmem, w);
+    if (warp == kSoftmaxWarps + 1) mma_issuer<D, BQ, BK, WRITE_MASK>(p, smem, bars, tmem, w);
     if (warp == kSoftmaxWarps + 3) s_waiter(p, bars, w);
   }
 

@@ -52,12 +52,9 @@ VPROD = WAIT + 2 * STEPS
 KPROD = VPROD + 2 * STEPS
 EPI = KPROD + STEPS
 # Warps of the roles: the softmax stamps come from warp 4s (the row-0 thread of
-# slot s), the S-wait and MMA stamps of slot s from its tensor-core warp 9 + 2s.
-K_WARP, V_WARP = 8, 10
-
-
-def mma_warp(s: int) -> int:
-    return 9 + 2 * s
+# slot s), the MMA stamps of both slots from the issuing warp 9 and the S-wait
+# stamps from the waiter warp 11.
+K_WARP, MMA_WARP, V_WARP, WAIT_WARP = 8, 9, 10, 11
 
 
 def load_trace_lib(path: str | None = None):
@@ -81,8 +78,8 @@ def phases(tr: np.ndarray, nblk: list[int]):
     for s in range(2):
         n = min(nblk[s], STEPS)
         sm = lambda j, e: int(tr[SOFTMAX + (s * STEPS + j) * 8 + e]) - off(4 * s)
-        mm = lambda j, e: int(tr[MMA + (s * STEPS + j) * 4 + e]) - off(mma_warp(s))
-        wt = lambda j: int(tr[WAIT + s * STEPS + j]) - off(mma_warp(s))
+        mm = lambda j, e: int(tr[MMA + (s * STEPS + j) * 4 + e]) - off(MMA_WARP)
+        wt = lambda j: int(tr[WAIT + s * STEPS + j]) - off(WAIT_WARP)
         for j in range(n):
             kept = tr[SOFTMAX + (s * STEPS + j) * 8 + 5] != 0
             ph = {"fence": sm(j, 1) - sm(j, 0), "load": sm(j, 2) - sm(j, 1), "max": sm(j, 3) - sm(j, 2),
