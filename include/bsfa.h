@@ -25,7 +25,8 @@
  * Thread safety: entry points may be called from several host threads; calls on
  * the same stream are ordered by the stream. The library allocates nothing per
  * call; it keeps one device status word per device (and, for bsfa_forward_host,
- * two copy streams and their events per device, created on first use).
+ * two copy streams, a second compute stream and their events per device,
+ * created on first use).
  *
  * The status word is shared by every kernel the library runs on a device,
  * whatever stream or host thread launched it: bsfa_get_status reports (and
@@ -142,12 +143,37 @@ bsfa_status bsfa_forward_heads(const void* q, const void* k, const void* v, cons
                                int kv_begin, int kv_count, void* stream);
 
 /*
+ * bsfa_forward_rows - bsfa_forward for query rows [row_begin, row_end) of every
+ * batch entry and head only. Every (query tile, key block) pair of those rows is
+ * computed exactly as the whole-layer call computes it ("Block Sparse Flash
+ * Attention" §4.4: query tiles are independent), so a layer can be computed in
+ * row chunks, e.g. while later rows are still being copied in. A chunk reads the
+ * K/V rows it attends to: [0, row_end) with the causal mask, all N without it.
+ * All tensors keep their full shapes and strides; only the selected rows of out
+ * and lse are written. The block mask, if given, is filled with 3 whole, then
+ * written for the selected query tiles.
+ *
+ *   row_begin   a multiple of 256, >= 0
+ *   row_end     row_begin < row_end <= N
+ *
+ * Else BSFA_ERR_INVALID_ARG; everything else as bsfa_forward.
+ */
+bsfa_status bsfa_forward_rows(const void* q, const void* k, const void* v, const float* tau, void* out, float* lse,
+                              uint8_t* block_mask, int B, int Hq, int Hkv, int N, int D, int Bq, int Bk, int causal,
+                              int row_begin, int row_end, void* stream);
+
+/*
  * bsfa_forward_host - bsfa_forward on HOST buffers, with the copies overlapped
- * with the kernel: the layer is cut into `chunks` runs of KV heads (as even as
- * Hkv allows); chunk c's Q/K/V go up on a copy stream, its heads are computed
- * (bsfa_forward_heads) once they have landed, and its out/lse rows come back on a
- * second copy stream while the next chunk computes. Asynchronous: everything is
- * done once `stream` reaches the call.
+ * with the kernel. K and V go up first, whole (one copy each). The query rows
+ * follow in `chunks` runs of whole 256-row units, the same rows of every batch
+ * entry, one copy per run; the runs shrink towards the end (cumulative share
+ * 1 - (1 - c/chunks)^2 after run c, at least one unit each), so little is left
+ * after the last upload. The kernel computes a run's rows (bsfa_forward_rows) as
+ * soon as they have landed, alternating between the caller's stream and a second
+ * compute stream, and the run's out rows come back on a second copy stream while
+ * the next run computes; lse (head-major, so a run's rows would be B * Hq short
+ * pieces) comes back whole after the last run. Asynchronous: everything is done
+ * once `stream` reaches the call.
  *
  *   q_host, k_host, v_host, tau_host   inputs in host memory, the layouts of
  *                                      bsfa_forward; page-locked (pinned) memory is
@@ -155,10 +181,10 @@ bsfa_status bsfa_forward_heads(const void* q, const void* k, const void* v, cons
  *   out_host, lse_host                 results in host memory (lse_host may be NULL)
  *   q_dev ... lse_dev                  device buffers of bsfa_forward's shapes, owned
  *                                      by the caller (lse_dev NULL iff lse_host is)
- *   chunks                             1 <= chunks <= min(Hkv, 64)
+ *   chunks                             1 <= chunks <= min(ceil(N / 256), 64)
  *
- * The library creates two copy streams and their events once per device and
- * reuses them; calls on one device share them: a call holds them (a host lock)
+ * The library creates two copy streams, a second compute stream and their
+ * events once per device and reuses them; calls on one device share them: a call holds them (a host lock)
  * while it enqueues, so concurrent calls from several host threads are
  * serialised and never consume each other's events.
  * Errors as bsfa_forward; BSFA_ERR_INVALID_ARG for a bad chunk count or a

@@ -137,11 +137,20 @@ def test_head_shard_entry_rejects_bad_ranges_without_touching_cuda(lib):
         assert "kv" in bsfa.bsfa_last_error().lower() or "heads" in bsfa.bsfa_last_error()
 
 
+def test_row_range_entry_rejects_bad_ranges_without_touching_cuda(lib):
+    call = lambda b, e: bsfa.bsfa_forward_rows(16, 16, 16, 16, 16, None, None, 1, 8, 4, 1000, 128, 128, 128, 1, b, e,
+                                               None)
+    for b, e in ((-256, 256), (128, 512), (256, 256), (512, 256), (0, 1001), (0, -1), (1024, 1000)):
+        assert call(b, e) == bsfa.BSFA_ERR_INVALID_ARG, (b, e)
+        assert "row" in bsfa.bsfa_last_error(), bsfa.bsfa_last_error()
+
+
 def test_host_buffer_entry_rejects_bad_arguments_without_touching_cuda(lib):
     ptrs = [16] * 12
     shape = (1, 8, 4, 512, 128, 128, 128, 1)
     assert bsfa.bsfa_forward_host(*ptrs, *shape, 0, None) == bsfa.BSFA_ERR_INVALID_ARG        # no chunks
-    assert bsfa.bsfa_forward_host(*ptrs, *shape, 5, None) == bsfa.BSFA_ERR_INVALID_ARG        # more chunks than KV heads
+    assert bsfa.bsfa_forward_host(*ptrs, *shape, 3, None) == bsfa.BSFA_ERR_INVALID_ARG        # more chunks than
+    assert "256" in bsfa.bsfa_last_error()                                                     # 256-row units
     missing = list(ptrs)
     missing[6] = None                                                                          # no device q
     assert bsfa.bsfa_forward_host(*missing, *shape, 2, None) == bsfa.BSFA_ERR_INVALID_ARG

@@ -226,20 +226,65 @@ def test_head_shards_equal_the_whole_layer(Hq, Hkv, shards):
     print(compare_tiles(x, tau, 128, 128, True, sharded, all_tiles(1, Hq, 1000, 128)).check())
 
 
+@pytest.mark.parametrize("Hq,Hkv,Bq,causal,cuts", [
+    (8, 4, 128, True, (0, 256, 768, 1000)),     # pairs of heads: 128-row units, a ragged last chunk
+    (8, 4, 64, False, (0, 512, 1000)),          # two query tiles per slot, bidirectional
+    (3, 1, 128, True, (0, 512, 1000)),          # odd group: pairs of adjacent tiles (256-row units)
+])
+def test_row_chunks_equal_the_whole_layer(Hq, Hkv, Bq, causal, cuts):
+    """Each row chunk (bsfa_forward_rows) writes exactly its rows, bit for bit what
+    the whole-layer call writes for them; later rows are left as they were. The
+    assembled chunks also match the oracle on every tile."""
+    N = 1000
+    cfg, x = _inputs(N, 128, Hq, Hkv, Bq, 128, causal, kind="planted", seed=80 + Hq)
+    tau = calibrate(x["q"], x["k"], Bq, 128, causal, [0.5])[0.5]
+    whole = run_gpu(x, tau, Bq, 128, causal)
+    from parity import to_device
+    q, k, v = (to_device(x[n]) for n in "qkv")
+    t = torch.tensor(np.asarray(tau, dtype=np.float32), device="cuda")
+    out = torch.full_like(q, 7.0)
+    lse = torch.full((1, Hq, N), 7.0, dtype=torch.float32, device="cuda")
+    mask = torch.empty_like(torch.from_numpy(whole["mask"]), device="cuda")
+    for r0, r1 in zip(cuts[:-1], cuts[1:]):
+        assert bsfa.bsfa_forward_rows(q, k, v, t, out, lse, mask, 1, Hq, Hkv, N, 128, Bq, 128, causal, r0, r1,
+                                      None) == bsfa.BSFA_OK
+        torch.cuda.synchronize()
+        o = out.float().cpu().numpy()
+        l = lse.cpu().numpy()
+        m = mask.cpu().numpy()
+        assert np.array_equal(o[:, :r1], whole["out"][:, :r1])
+        assert np.array_equal(l[:, :, :r1], whole["lse"][:, :, :r1])
+        t0, t1 = r0 // Bq, -(-r1 // Bq)
+        assert np.array_equal(m[:, :, t0:t1], whole["mask"][:, :, t0:t1])    # this chunk's tiles; the rest hold 3
+        assert (m[:, :, :t0] == 3).all() and (m[:, :, t1:] == 3).all()
+        if r1 < N:
+            assert (o[:, r1:] == 7.0).all()
+    assert bsfa.bsfa_get_status(None) == bsfa.BSFA_OK
+    chunked = {"out": o.astype(np.float64), "lse": l.astype(np.float64), "mask": whole["mask"]}
+    print(compare_tiles(x, tau, Bq, 128, causal, chunked, all_tiles(1, Hq, N, Bq)).check())
+
+
 # ----------------------------------------------------------------------------- host buffers, overlapped copies
 
-@pytest.mark.parametrize("chunks", [1, 3, 4])
-def test_host_buffer_call_equals_the_device_call(chunks):
-    """bsfa_forward_host (copies in runs of KV heads, overlapped with the kernel)
-    returns exactly what the device call computes, for an uneven chunk split and a
-    ragged N, and matches the oracle on every tile."""
-    cfg, x = _inputs(900, 128, 8, 4, 128, 64, True, kind="planted", seed=70)
-    tau = calibrate(x["q"], x["k"], 128, 64, True, [0.5])[0.5]
-    dev = run_gpu(x, tau, 128, 64, True, want_mask=True)
+@pytest.mark.parametrize("B,Hq,Hkv,N,causal,chunks", [
+    (1, 8, 4, 900, True, 1),       # one chunk: the plain call
+    (1, 8, 4, 900, True, 3),       # uneven 256-row split, ragged N
+    (1, 8, 4, 900, True, 4),       # one 256-row unit per chunk, the last one ragged
+    (2, 8, 4, 900, False, 3),      # bidirectional: K and V go up first; two batch entries
+    (2, 3, 1, 700, True, 2),       # odd group size: CTAs pair adjacent row tiles (256-row units)
+])
+def test_host_buffer_call_equals_the_device_call(B, Hq, Hkv, N, causal, chunks):
+    """bsfa_forward_host (copies in chunks of query rows, overlapped with the
+    kernel) returns exactly what the device call computes, for uneven chunk splits,
+    a ragged N, several batch entries and both masks, and matches the oracle on
+    every tile."""
+    cfg, x = _inputs(N, 128, Hq, Hkv, 128, 64, causal, kind="planted", seed=70, B=B)
+    tau = calibrate(x["q"], x["k"], 128, 64, causal, [0.5])[0.5]
+    dev = run_gpu(x, tau, 128, 64, causal, want_mask=True)
     host = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).pin_memory()
     q, k, v = (host(x[n]) for n in "qkv")
     t = torch.tensor(np.asarray(tau, dtype=np.float32)).pin_memory()
-    out, lse = bsfa.forward_host(q, k, v, t, Bq=128, Bk=64, causal=True, chunks=chunks)
+    out, lse = bsfa.forward_host(q, k, v, t, Bq=128, Bk=64, causal=causal, chunks=chunks)
     assert bsfa.bsfa_get_status(None) == bsfa.BSFA_OK
     host_res = {"out": out.float().numpy().astype(np.float64), "lse": lse.numpy().astype(np.float64),
                 "mask": dev["mask"]}
@@ -247,7 +292,7 @@ def test_host_buffer_call_equals_the_device_call(chunks):
     assert np.array_equal(host_res["lse"], dev["lse"])
     # The host call's own output against the oracle (the mask comes from the device
     # call, which the bit-equality above ties to the host call's result).
-    print(compare_tiles(x, tau, 128, 64, True, host_res, all_tiles(1, 8, 900, 128)).check())
+    print(compare_tiles(x, tau, 128, 64, causal, host_res, all_tiles(B, Hq, N, 128)).check())
 
 
 # ----------------------------------------------------------------------------- the largest supported length

@@ -6,7 +6,7 @@ fallback: if the library is missing or the device is not sm_100, calls fail
 loudly.
 
 The functions named like the C entry points (``bsfa_forward``,
-``bsfa_forward_tau_table``, ``bsfa_forward_gap``, ``bsfa_forward_heads``, ``bsfa_forward_host``,
+``bsfa_forward_tau_table``, ``bsfa_forward_gap``, ``bsfa_forward_heads``, ``bsfa_forward_rows``, ``bsfa_forward_host``,
 ``bsfa_forward_varlen``, ``bsfa_validate``,
 ``bsfa_get_status``, ``bsfa_get_debug_counts``,
 ``bsfa_selftest_lost_arrival``, ``bsfa_status_string``, ``bsfa_last_error``)
@@ -28,7 +28,8 @@ BSFA_ERR_UNSUPPORTED = 2
 BSFA_ERR_CUDA = 3
 BSFA_ERR_DEVICE_TIMEOUT = 4
 
-EXPORTED = ("bsfa_forward", "bsfa_forward_tau_table", "bsfa_forward_gap", "bsfa_forward_heads", "bsfa_forward_host",
+EXPORTED = ("bsfa_forward", "bsfa_forward_tau_table", "bsfa_forward_gap", "bsfa_forward_heads", "bsfa_forward_rows",
+            "bsfa_forward_host",
             "bsfa_forward_varlen", "bsfa_validate", "bsfa_get_status", "bsfa_get_debug_counts",
             "bsfa_selftest_lost_arrival", "bsfa_status_string", "bsfa_last_error")
 
@@ -58,6 +59,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.bsfa_forward_gap.restype = i
     lib.bsfa_forward_heads.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, i, vp]
     lib.bsfa_forward_heads.restype = i
+    lib.bsfa_forward_rows.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, i, vp]
+    lib.bsfa_forward_rows.restype = i
     lib.bsfa_forward_host.argtypes = [vp] * 12 + [i] * 9 + [vp]
     lib.bsfa_forward_host.restype = i
     lib.bsfa_forward_varlen.argtypes = [vp, vp, vp, vp, i, i, vp, vp, vp, vp, i, i, i, i, i, i, i, vp]
@@ -111,6 +114,13 @@ def bsfa_forward_tau_table(q, k, v, tau_table, tau_tiles, out, lse, block_mask, 
 def bsfa_forward_gap(q, k, v, gamma, out, lse, block_mask, B, Hq, Hkv, N, D, Bq, Bk, causal, stream) -> int:
     return load().bsfa_forward_gap(_ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(out), _ptr(lse), _ptr(block_mask),
                                    B, Hq, Hkv, N, D, Bq, Bk, int(bool(causal)), _stream(stream))
+
+
+def bsfa_forward_rows(q, k, v, tau, out, lse, block_mask, B, Hq, Hkv, N, D, Bq, Bk, causal, row_begin, row_end,
+                      stream) -> int:
+    return load().bsfa_forward_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(tau), _ptr(out), _ptr(lse), _ptr(block_mask),
+                                    B, Hq, Hkv, N, D, Bq, Bk, int(bool(causal)), int(row_begin), int(row_end),
+                                    _stream(stream))
 
 
 def bsfa_forward_heads(q, k, v, tau, out, lse, block_mask, B, Hq, Hkv, N, D, Bq, Bk, causal, kv_begin, kv_count,
@@ -256,7 +266,8 @@ def forward_host(q, k, v, tau, *, Bq: int, Bk: int, causal: bool, device=None, s
     q, k, v: bf16 CPU tensors (pinned for asynchronous copies); tau: fp32 CPU tensor, [Hq] or [Hq, T].
     ``bufs`` (from ``device_buffers``) holds reusable device and pinned host buffers.
     With one threshold per head this is ``bsfa_forward_host``: the copies run in
-    ``chunks`` runs of KV heads (default min(Hkv, 8)) overlapped with the kernel.
+    ``chunks`` runs of query rows (whole 256-row units, shrinking towards the end;
+    default min(ceil(N/256), 8)) overlapped with the kernel.
     Other gates copy, run and copy back in turn on ``stream``.
     Returns (out_host, lse_host).
     """
@@ -272,7 +283,7 @@ def forward_host(q, k, v, tau, *, Bq: int, Bk: int, causal: bool, device=None, s
         Hkv = k.shape[2]
         _check(bsfa_forward_host(q, k, v, tau, bufs["out_host"], bufs["lse_host"], bufs["q"], bufs["k"], bufs["v"],
                                  bufs["tau"], bufs["out"], bufs["lse"], B, Hq, Hkv, N, D, Bq, Bk, causal,
-                                 chunks or min(Hkv, 8), stream))
+                                 chunks or min(-(-N // 256), 8), stream))
         stream.synchronize()
         return bufs["out_host"], bufs["lse_host"]
     with torch.cuda.stream(stream):

@@ -1,6 +1,7 @@
 // C ABI of the BSFA prefill forward: argument validation, TMA descriptor
 // encoding, kernel dispatch and the device status word. The declarations and
 // their contracts are in include/bsfa.h.
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -150,7 +151,7 @@ namespace {
 bsfa_status forward_impl(const void* q, const void* k, const void* v, const float* tau, int tau_tiles, int gate_gap,
                          void* out, float* lse, uint8_t* block_mask, int B, int Hq, int Hkv, int N, int D, int Bq,
                          int Bk, int causal, void* stream, const int* cu_seqlens = nullptr, int max_seqlen = 0,
-                         int kv_begin = 0, int kv_count = -1) {
+                         int kv_begin = 0, int kv_count = -1, int row_begin = 0, int row_end = -1) {
   bsfa_status st;
   if (cu_seqlens) {
     // Packed sequences: the key-block limit (the per-CTA gate decisions) applies
@@ -173,6 +174,11 @@ bsfa_status forward_impl(const void* q, const void* k, const void* v, const floa
   if (kv_count < 0) kv_count = Hkv;
   if (kv_begin < 0 || kv_count <= 0 || kv_begin + kv_count > Hkv)
     return fail(BSFA_ERR_INVALID_ARG, "KV heads [%d, %d) are not inside [0, %d)", kv_begin, kv_begin + kv_count, Hkv);
+  if (row_end < 0) row_end = max_seqlen;
+  if (row_begin < 0 || row_begin % 256 != 0 || row_end <= row_begin || row_end > max_seqlen ||
+      (cu_seqlens && (row_begin != 0 || row_end != max_seqlen)))
+    return fail(BSFA_ERR_INVALID_ARG, "query rows [%d, %d) are not a 256-aligned range inside [0, %d)", row_begin,
+                row_end, max_seqlen);
   if (tau_tiles < 0) return fail(BSFA_ERR_INVALID_ARG, "tau_tiles=%d is negative", tau_tiles);
   if (!q || !k || !v || !tau || !out) return fail(BSFA_ERR_INVALID_ARG, "q, k, v, tau and out must be non-null");
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16))
@@ -231,8 +237,11 @@ bsfa_status forward_impl(const void* q, const void* k, const void* v, const floa
 #endif
   p.scale = (float)(1.0 / std::sqrt((double)D));
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
-  const int tiles = (max_seqlen + 127) / 128;
-  const int grid = p.pair_heads ? B * (p.hq_count / 2) * tiles : B * p.hq_count * ((tiles + 1) / 2);
+  // Row units: 128-row tiles when a CTA pairs two heads, else pairs of adjacent tiles.
+  const int unit_rows = p.pair_heads ? 128 : 256;
+  p.row_unit0 = row_begin / unit_rows;
+  p.row_units = (row_end + unit_rows - 1) / unit_rows - p.row_unit0;
+  const int grid = (p.pair_heads ? B * (p.hq_count / 2) : B * p.hq_count) * p.row_units;
   e = (D == 64) ? bsfa::launch_fwd_d64(tq, tk, tv, p, Bq, Bk, causal != 0, block_mask != nullptr, grid, dev, s)
                 : bsfa::launch_fwd_d128(tq, tk, tv, p, Bq, Bk, causal != 0, block_mask != nullptr, grid, dev, s);
   if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
@@ -246,7 +255,7 @@ bsfa_status forward_impl(const void* q, const void* k, const void* v, const floa
 // (their copies are serialised).
 constexpr int kMaxChunks = 64;
 struct HostPipe {
-  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaStream_t h2d = nullptr, d2h = nullptr, aux = nullptr;   // aux: a second compute stream
   cudaEvent_t start = nullptr, in[kMaxChunks] = {}, done[kMaxChunks] = {}, out = nullptr;
   std::mutex call;
 };
@@ -256,6 +265,7 @@ std::mutex g_pipe_mutex;
 void destroy_pipe_parts(HostPipe& t) {
   if (t.h2d) cudaStreamDestroy(t.h2d);
   if (t.d2h) cudaStreamDestroy(t.d2h);
+  if (t.aux) cudaStreamDestroy(t.aux);
   if (t.start) cudaEventDestroy(t.start);
   if (t.out) cudaEventDestroy(t.out);
   for (int c = 0; c < kMaxChunks; ++c) {
@@ -273,6 +283,7 @@ bsfa_status host_pipe(int dev, HostPipe** pipe) {
     HostPipe t;
     cudaError_t e = cudaStreamCreateWithFlags(&t.h2d, cudaStreamNonBlocking);
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&t.d2h, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&t.aux, cudaStreamNonBlocking);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&t.start, cudaEventDisableTiming);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&t.out, cudaEventDisableTiming);
     for (int c = 0; c < kMaxChunks && e == cudaSuccess; ++c) {
@@ -284,6 +295,7 @@ bsfa_status host_pipe(int dev, HostPipe** pipe) {
       return cuda_fail(e, "creating the copy streams");
     }
     hp.d2h = t.d2h;
+    hp.aux = t.aux;
     hp.start = t.start;
     hp.out = t.out;
     for (int c = 0; c < kMaxChunks; ++c) {
@@ -296,13 +308,18 @@ bsfa_status host_pipe(int dev, HostPipe** pipe) {
   return BSFA_OK;
 }
 
-// Rows [0, rows) of a row-major [rows, cols_total] array of `elem`-byte
-// elements, columns [col0, col0 + cols): one strided copy.
-cudaError_t copy_cols(void* dst, const void* src, size_t rows, size_t cols_total, size_t col0, size_t cols, size_t elem,
-                      cudaMemcpyKind kind, cudaStream_t st) {
-  const size_t pitch = cols_total * elem;
-  return cudaMemcpy2DAsync(static_cast<char*>(dst) + col0 * elem, pitch, static_cast<const char*>(src) + col0 * elem,
-                           pitch, cols * elem, rows, kind, st);
+// Rows [r0, r1) of every batch entry of a [B, N, row_bytes] array: one copy
+// (B strided pieces of contiguous rows, or one contiguous run when they touch).
+cudaError_t copy_rows(void* dst, const void* src, int B, int N, size_t row_bytes, int r0, int r1, cudaMemcpyKind kind,
+                      cudaStream_t st) {
+  const size_t pitch = (size_t)N * row_bytes;
+  if (B == 1 || (r0 == 0 && r1 == N))
+    return cudaMemcpyAsync(static_cast<char*>(dst) + (size_t)r0 * row_bytes,
+                           static_cast<const char*>(src) + (size_t)r0 * row_bytes,
+                           (size_t)(r1 - r0) * row_bytes + (size_t)(B - 1) * pitch, kind, st);
+  return cudaMemcpy2DAsync(static_cast<char*>(dst) + (size_t)r0 * row_bytes, pitch,
+                           static_cast<const char*>(src) + (size_t)r0 * row_bytes, pitch, (size_t)(r1 - r0) * row_bytes,
+                           (size_t)B, kind, st);
 }
 
 }  // namespace
@@ -339,6 +356,14 @@ bsfa_status bsfa_forward_heads(const void* q, const void* k, const void* v, cons
                       kv_begin, kv_count);
 }
 
+bsfa_status bsfa_forward_rows(const void* q, const void* k, const void* v, const float* tau, void* out, float* lse,
+                              uint8_t* block_mask, int B, int Hq, int Hkv, int N, int D, int Bq, int Bk, int causal,
+                              int row_begin, int row_end, void* stream) {
+  if (row_end < 0) return fail(BSFA_ERR_INVALID_ARG, "row_end=%d is negative", row_end);
+  return forward_impl(q, k, v, tau, 0, 0, out, lse, block_mask, B, Hq, Hkv, N, D, Bq, Bk, causal, stream, nullptr, 0,
+                      0, -1, row_begin, row_end);
+}
+
 bsfa_status bsfa_forward_host(const void* q_host, const void* k_host, const void* v_host, const float* tau_host,
                               void* out_host, float* lse_host, void* q_dev, void* k_dev, void* v_dev, float* tau_dev,
                               void* out_dev, float* lse_dev, int B, int Hq, int Hkv, int N, int D, int Bq, int Bk,
@@ -349,8 +374,9 @@ bsfa_status bsfa_forward_host(const void* q_host, const void* k_host, const void
     return fail(BSFA_ERR_INVALID_ARG, "host and device q, k, v, tau and out must be non-null");
   if ((lse_host == nullptr) != (lse_dev == nullptr))
     return fail(BSFA_ERR_INVALID_ARG, "lse needs both a host and a device buffer, or neither");
-  if (chunks < 1 || chunks > Hkv || chunks > kMaxChunks)
-    return fail(BSFA_ERR_INVALID_ARG, "chunks=%d must be in [1, min(Hkv=%d, %d)]", chunks, Hkv, kMaxChunks);
+  const int units = (N + 255) / 256;          // chunk boundaries fall on 256-row multiples
+  if (chunks < 1 || chunks > units || chunks > kMaxChunks)
+    return fail(BSFA_ERR_INVALID_ARG, "chunks=%d must be in [1, min(ceil(N/256)=%d, %d)]", chunks, units, kMaxChunks);
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
@@ -360,39 +386,50 @@ bsfa_status bsfa_forward_host(const void* q_host, const void* k_host, const void
   if (st != BSFA_OK) return st;
   std::lock_guard<std::mutex> call_lock(hp->call);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int group = Hq / Hkv;
-  const size_t rows = (size_t)B * N;
+  const size_t q_row = (size_t)Hq * D * 2, kv_row = (size_t)Hkv * D * 2;
   // The copies start once earlier work on the caller's stream is done.
   e = cudaEventRecord(hp->start, s);
   if (e == cudaSuccess) e = cudaStreamWaitEvent(hp->h2d, hp->start, 0);
   if (e == cudaSuccess) e = cudaMemcpyAsync(tau_dev, tau_host, (size_t)Hq * sizeof(float), cudaMemcpyHostToDevice, hp->h2d);
+  // K and V go up first, whole (one copy each); then the query rows in chunks,
+  // one copy each. A chunk needs its own Q rows and the keys it attends to, all
+  // of which have landed by then.
+  if (e == cudaSuccess) e = copy_rows(k_dev, k_host, B, N, kv_row, 0, N, cudaMemcpyHostToDevice, hp->h2d);
+  if (e == cudaSuccess) e = copy_rows(v_dev, v_host, B, N, kv_row, 0, N, cudaMemcpyHostToDevice, hp->h2d);
   if (e != cudaSuccess) return cuda_fail(e, "host pipeline start");
+  int u_prev = 0;
   for (int c = 0; c < chunks; ++c) {
-    // Chunk c: KV heads [g0, g1) and their query heads, as even a split as Hkv allows.
-    const int g0 = (int)((long long)Hkv * c / chunks), g1 = (int)((long long)Hkv * (c + 1) / chunks);
-    const int h0 = g0 * group, nh = (g1 - g0) * group;
-    e = copy_cols(q_dev, q_host, rows, (size_t)Hq * D, (size_t)h0 * D, (size_t)nh * D, 2, cudaMemcpyHostToDevice, hp->h2d);
-    if (e == cudaSuccess)
-      e = copy_cols(k_dev, k_host, rows, (size_t)Hkv * D, (size_t)g0 * D, (size_t)(g1 - g0) * D, 2,
-                    cudaMemcpyHostToDevice, hp->h2d);
-    if (e == cudaSuccess)
-      e = copy_cols(v_dev, v_host, rows, (size_t)Hkv * D, (size_t)g0 * D, (size_t)(g1 - g0) * D, 2,
-                    cudaMemcpyHostToDevice, hp->h2d);
+    // Chunk c: query rows [r0, r1) of every batch entry, in whole 256-row units.
+    // The chunks shrink towards the end (cumulative share 1 - (1 - (c+1)/chunks)^2,
+    // at least one unit each): what is left after the last upload (the last
+    // chunk's compute and its copy back) is then short.
+    const double f = 1.0 - (1.0 - (double)(c + 1) / chunks) * (1.0 - (double)(c + 1) / chunks);
+    int u1 = (c + 1 == chunks) ? units : (int)(units * f + 0.5);
+    u1 = std::max(u1, u_prev + 1);
+    u1 = std::min(u1, units - (chunks - 1 - c));
+    const int r0 = u_prev * 256, r1 = std::min(u1 * 256, N);
+    u_prev = u1;
+    e = copy_rows(q_dev, q_host, B, N, q_row, r0, r1, cudaMemcpyHostToDevice, hp->h2d);
     if (e == cudaSuccess) e = cudaEventRecord(hp->in[c], hp->h2d);
-    if (e == cudaSuccess) e = cudaStreamWaitEvent(s, hp->in[c], 0);
+    // Chunks alternate between the caller's stream and a second compute stream:
+    // a late chunk has few CTAs, each as long as the longest causal row, so two
+    // of them run side by side.
+    cudaStream_t cs = (c % 2 == 0) ? s : hp->aux;
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(cs, hp->in[c], 0);
     if (e != cudaSuccess) return cuda_fail(e, "host-to-device copy");
     st = forward_impl(q_dev, k_dev, v_dev, tau_dev, 0, 0, out_dev, lse_dev, nullptr, B, Hq, Hkv, N, D, Bq, Bk, causal,
-                      stream, nullptr, 0, g0, g1 - g0);
+                      cs, nullptr, 0, 0, Hkv, r0, r1);
     if (st != BSFA_OK) return st;
-    e = cudaEventRecord(hp->done[c], s);
+    e = cudaEventRecord(hp->done[c], cs);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(hp->d2h, hp->done[c], 0);
-    if (e == cudaSuccess)
-      e = copy_cols(out_host, out_dev, rows, (size_t)Hq * D, (size_t)h0 * D, (size_t)nh * D, 2, cudaMemcpyDeviceToHost,
-                    hp->d2h);
-    if (e == cudaSuccess && lse_host)   // lse [B, Hq, N]: the chunk's heads are nh * N floats per batch entry
-      e = copy_cols(lse_host, lse_dev, (size_t)B, (size_t)Hq * N, (size_t)h0 * N, (size_t)nh * N, 4,
-                    cudaMemcpyDeviceToHost, hp->d2h);
+    if (e == cudaSuccess) e = copy_rows(out_host, out_dev, B, N, q_row, r0, r1, cudaMemcpyDeviceToHost, hp->d2h);
     if (e != cudaSuccess) return cuda_fail(e, "device-to-host copy");
+  }
+  // lse [B, Hq, N] is head-major: a chunk's rows are B * Hq short runs, so it comes
+  // back whole, in one copy, behind the last chunk.
+  if (lse_host) {
+    e = cudaMemcpyAsync(lse_host, lse_dev, (size_t)B * Hq * N * sizeof(float), cudaMemcpyDeviceToHost, hp->d2h);
+    if (e != cudaSuccess) return cuda_fail(e, "device-to-host copy (lse)");
   }
   // The caller's stream reaches the end of the call once the last result is on the host.
   e = cudaEventRecord(hp->out, hp->d2h);

@@ -61,6 +61,9 @@ struct FwdParams {
   int group;          // Hq / Hkv
   int hq_begin, hq_count;   // the query heads this launch computes (all of them unless head-sharded)
   int pair_heads;     // 1: slots are query heads 2p and 2p+1 on the same rows
+  // The query rows this launch computes, in row units (128-row tiles when
+  // pair_heads, else pairs of adjacent 128-row tiles): [row_unit0, row_unit0 + row_units).
+  int row_unit0, row_units;
   int gate_gap;       // 0: the BSFA gate (block maximum against tau); 1: the gap gate, tau holding gamma
                       // (selects the kernel's GAP template argument at launch)
   float scale;        // 1/sqrt(D): the gate compares s_max(raw) * scale against tau
@@ -194,23 +197,21 @@ struct SeqSpan {
 
 template <bool VARLEN>
 __device__ __forceinline__ FwdUnit decode_unit(const FwdParams& p, int u, bool causal, int bk, SeqSpan& sp) {
-  const int tiles = ((VARLEN ? p.max_seqlen : p.N) + 127) / 128;
   FwdUnit w;
   if (p.pair_heads) {
     // Consecutive units: the head pairs of one row block, a KV group's pairs adjacent.
     const int per = p.B * (p.hq_count / 2);
     const int hp = u % per, t = u / per;
-    const int qt = causal ? tiles - 1 - t : t;     // heaviest causal rows first
+    const int qt = p.row_unit0 + (causal ? p.row_units - 1 - t : t);   // heaviest causal rows first
     w.b = hp / (p.hq_count / 2);
     const int h0 = p.hq_begin + 2 * (hp % (p.hq_count / 2));
     w.hq[0] = h0;
     w.hq[1] = h0 + 1;
     w.q0[0] = w.q0[1] = qt * 128;
   } else {
-    const int pairs = (tiles + 1) / 2;
     const int per = p.B * p.hq_count;
     const int bh = u % per, t = u / per;
-    const int qp = causal ? pairs - 1 - t : t;
+    const int qp = p.row_unit0 + (causal ? p.row_units - 1 - t : t);
     w.b = bh / p.hq_count;
     w.hq[0] = w.hq[1] = p.hq_begin + bh % p.hq_count;
     w.q0[0] = 2 * qp * 128;
