@@ -61,6 +61,9 @@ def parse():
     ap.add_argument("--tau-table", type=int, default=None, metavar="K",
                     help="gate with the stored per-position (fixed-k) table level that keeps K blocks per tile")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU-oracle baseline")
+    ap.add_argument("--cpu-tiles", type=int, default=None,
+                    help="run the CPU-oracle baseline on exactly this many seeded query tiles (no time budget) and "
+                         "extrapolate to the full layer; default 64 for c4, else the --cpu-seconds budget")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-sweep", action="store_true",
                     help="leave out the skip sweep (the default c2 line also times the 32K layer at 30/50/70/90%% "
@@ -522,13 +525,28 @@ def run_ours(args):
         dist.destroy_process_group()
     if rank == 0:
         if world == 1:
-            budget = args.cpu_seconds
-            tiles = sample_tiles(cfg, 4096, seed=cfg.seed + 5)
-            np.random.default_rng(0).shuffle(tiles)
-            f, t, n = oracle_sample(cfg, x, taus, budget, tiles, args.gate)
-            line["cpu_baseline"] = {"value": f / t / 1e12, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
-                                    "sample": f"{n} seeded query tiles of {cfg.name} (about {t:.1f} s of oracle "
-                                              f"work), dense-equivalent FLOPs of those tiles"}
+            count = args.cpu_tiles if args.cpu_tiles is not None else (64 if cfg.name == "c4" else 0)
+            if count > 0:
+                # An exact seeded sample (spread over heads, the first and last tile of
+                # head 0 among them), extrapolated to the layer by dense-equivalent FLOPs.
+                tiles = sample_tiles(cfg, count, seed=cfg.seed + 5)
+                f, t, n = oracle_sample(cfg, x, taus, float("inf"), tiles, args.gate)
+                layer_s = layer_dense_flops / (f / t)
+                line["cpu_baseline"] = {"value": f / t / 1e12, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+                                        "sample": f"{n} seeded query tiles of {cfg.name} (exact count, {t:.1f} s of "
+                                                  f"oracle work), dense-equivalent FLOPs of those tiles",
+                                        "seconds_per_tile": t / n,
+                                        "extrapolated_layer_s": layer_s,
+                                        "extrapolated": "full-layer time = the layer's dense-equivalent FLOPs / "
+                                                        "the sample's FLOP rate"}
+            else:
+                budget = args.cpu_seconds
+                tiles = sample_tiles(cfg, 4096, seed=cfg.seed + 5)
+                np.random.default_rng(0).shuffle(tiles)
+                f, t, n = oracle_sample(cfg, x, taus, budget, tiles, args.gate)
+                line["cpu_baseline"] = {"value": f / t / 1e12, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+                                        "sample": f"{n} seeded query tiles of {cfg.name} (about {t:.1f} s of oracle "
+                                                  f"work), dense-equivalent FLOPs of those tiles"}
         print(json.dumps(line), flush=True)
     return 0
 
