@@ -146,6 +146,30 @@ def oracle_sample(cfg, x, taus, budget_s, tiles, gate="tau"):
     return flops, time.perf_counter() - t0, done
 
 
+def cpu_baseline(cfg, x, taus, gate, layer_dense_flops, count, budget_s):
+    """The oracle timed on the host cores: the bench line's cpu_baseline object.
+
+    count > 0: exactly that many seeded query tiles (spread over heads, the first
+    and last tile of head 0 among them), no time budget, extrapolated to the
+    layer by dense-equivalent FLOPs. Otherwise: shuffled seeded tiles until
+    budget_s seconds of oracle work are spent."""
+    if count > 0:
+        tiles = sample_tiles(cfg, count, seed=cfg.seed + 5)
+        f, t, n = oracle_sample(cfg, x, taus, float("inf"), tiles, gate)
+        return {"value": f / t / 1e12, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+                "sample": f"{n} seeded query tiles of {cfg.name} (exact count, {t:.1f} s of oracle work), "
+                          f"dense-equivalent FLOPs of those tiles",
+                "seconds_per_tile": t / n,
+                "extrapolated_layer_s": layer_dense_flops / (f / t),
+                "extrapolated": "full-layer time = the layer's dense-equivalent FLOPs / the sample's FLOP rate"}
+    tiles = sample_tiles(cfg, 4096, seed=cfg.seed + 5)
+    np.random.default_rng(0).shuffle(tiles)
+    f, t, n = oracle_sample(cfg, x, taus, budget_s, tiles, gate)
+    return {"value": f / t / 1e12, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+            "sample": f"{n} seeded query tiles of {cfg.name} (about {t:.1f} s of oracle work), "
+                      f"dense-equivalent FLOPs of those tiles"}
+
+
 def head_shard(rank: int, world: int, Hkv: int) -> tuple[int, int]:
     """(first KV head, KV head count) of ``rank`` when a layer's KV groups are split
     evenly across ``world`` ranks."""
@@ -526,27 +550,7 @@ def run_ours(args):
     if rank == 0:
         if world == 1:
             count = args.cpu_tiles if args.cpu_tiles is not None else (64 if cfg.name == "c4" else 0)
-            if count > 0:
-                # An exact seeded sample (spread over heads, the first and last tile of
-                # head 0 among them), extrapolated to the layer by dense-equivalent FLOPs.
-                tiles = sample_tiles(cfg, count, seed=cfg.seed + 5)
-                f, t, n = oracle_sample(cfg, x, taus, float("inf"), tiles, args.gate)
-                layer_s = layer_dense_flops / (f / t)
-                line["cpu_baseline"] = {"value": f / t / 1e12, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
-                                        "sample": f"{n} seeded query tiles of {cfg.name} (exact count, {t:.1f} s of "
-                                                  f"oracle work), dense-equivalent FLOPs of those tiles",
-                                        "seconds_per_tile": t / n,
-                                        "extrapolated_layer_s": layer_s,
-                                        "extrapolated": "full-layer time = the layer's dense-equivalent FLOPs / "
-                                                        "the sample's FLOP rate"}
-            else:
-                budget = args.cpu_seconds
-                tiles = sample_tiles(cfg, 4096, seed=cfg.seed + 5)
-                np.random.default_rng(0).shuffle(tiles)
-                f, t, n = oracle_sample(cfg, x, taus, budget, tiles, args.gate)
-                line["cpu_baseline"] = {"value": f / t / 1e12, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
-                                        "sample": f"{n} seeded query tiles of {cfg.name} (about {t:.1f} s of oracle "
-                                                  f"work), dense-equivalent FLOPs of those tiles"}
+            line["cpu_baseline"] = cpu_baseline(cfg, x, taus, args.gate, layer_dense_flops, count, args.cpu_seconds)
         print(json.dumps(line), flush=True)
     return 0
 
